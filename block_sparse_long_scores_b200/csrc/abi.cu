@@ -1,0 +1,333 @@
+// abi.cu -- the C ABI of include/msa.h: argument checks, workspace sizing, TMA tensor-map
+// encoding and kernel launches.  Nothing here allocates memory; every launch goes to the
+// caller's stream and no call synchronises the host.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "launch.cuh"
+#include "msa.h"
+
+
+using namespace msa;
+
+namespace {
+
+std::atomic<int64_t> g_launches{0};
+
+// ------------------------------------------------------------------ driver entry point (TMA)
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle; dims innermost first; strides (bytes) of dims 1..rank-1.
+bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, const uint64_t *strides,
+              const uint32_t *box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gd[5], gs[4];
+    cuuint32_t bx[5], es[5];
+    for (int r = 0; r < rank; ++r) {
+        gd[r] = dims[r];
+        bx[r] = box[r];
+        es[r] = 1;
+        if (r + 1 < rank) gs[r] = strides[r];
+    }
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), gd, gs, bx, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+// --------------------------------------------------------------------------- validation
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+msa_status_t check_cfg(const msa_config_t *c) {
+    if (!c) return MSA_ERR_INVALID_ARG;
+    if (c->num_q_heads <= 0 || c->num_kv_heads <= 0 || c->num_q_heads % c->num_kv_heads) return MSA_ERR_INVALID_ARG;
+    const int G = c->num_q_heads / c->num_kv_heads;
+    if (c->n_topk < 0 || (c->use_sink != 0 && c->use_sink != 1)) return MSA_ERR_INVALID_ARG;
+    if (!(c->softmax_scale >= 0.f) || std::isinf(c->softmax_scale)) return MSA_ERR_INVALID_ARG;
+    if (c->head_dim != 64 && c->head_dim != 128) return MSA_ERR_UNSUPPORTED;
+    if (c->block_size != 64 && c->block_size != 128) return MSA_ERR_UNSUPPORTED;
+    if (c->index_dim != 64) return MSA_ERR_UNSUPPORTED;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return MSA_ERR_UNSUPPORTED;
+    if (c->n_topk + 1 + c->use_sink > 256) return MSA_ERR_UNSUPPORTED;
+    return MSA_OK;
+}
+
+msa_status_t check_shape(const msa_config_t *c, const msa_shape_t *s) {
+    if (!s) return MSA_ERR_INVALID_ARG;
+    if (s->batch <= 0 || s->max_seqlen <= 0 || s->total_rows < 0) return MSA_ERR_INVALID_ARG;
+    const int64_t need_blocks = (s->max_seqlen + c->block_size - 1) / c->block_size;
+    if (s->mode == MSA_PREFILL) {
+        if (!s->cu_seqlens || !s->cu_blocks) return MSA_ERR_INVALID_ARG;
+        if (s->total_blocks < 0 || s->max_blocks != need_blocks) return MSA_ERR_INVALID_ARG;
+        if (s->total_rows >= (int64_t)1 << 31 || s->total_blocks >= (int64_t)1 << 31) return MSA_ERR_UNSUPPORTED;
+    } else if (s->mode == MSA_DECODE) {
+        if (!s->seqlens || s->total_rows != s->batch || s->max_blocks < need_blocks) return MSA_ERR_INVALID_ARG;
+        if ((int64_t)s->batch * c->num_kv_heads * s->max_seqlen >= (int64_t)1 << 31) return MSA_ERR_UNSUPPORTED;
+    } else {
+        return MSA_ERR_INVALID_ARG;
+    }
+    if (s->max_blocks > 32768) return MSA_ERR_UNSUPPORTED;
+    return MSA_OK;
+}
+
+Prob make_prob(const msa_config_t *c, const msa_shape_t *s, int64_t rb, int64_t re, int32_t *err) {
+    Prob P{};
+    P.mode = s->mode;
+    P.batch = s->batch;
+    P.Hq = c->num_q_heads;
+    P.Hkv = c->num_kv_heads;
+    P.G = P.Hq / P.Hkv;
+    P.D = c->head_dim;
+    P.B = c->block_size;
+    P.d = c->index_dim;
+    P.n_topk = c->n_topk;
+    P.use_sink = c->use_sink;
+    P.k_tot = c->n_topk + 1 + c->use_sink;
+    P.scale = c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / std::sqrt((float)c->head_dim);
+    P.scale_log2 = P.scale * 1.4426950408889634f;
+    P.T = s->total_rows;
+    P.total_blocks = s->mode == MSA_PREFILL ? s->total_blocks : 0;
+    P.Lmax = s->mode == MSA_DECODE ? s->max_seqlen : 0;
+    P.max_blocks = s->max_blocks;
+    P.cu_seqlens = s->cu_seqlens;
+    P.cu_blocks = s->cu_blocks;
+    P.seqlens = s->seqlens;
+    P.row_begin = rb;
+    P.row_end = re;
+    P.err = err;
+    return P;
+}
+
+msa_status_t cuda_status(cudaError_t e, int kernels) {
+    if (e != cudaSuccess) return MSA_ERR_CUDA;
+    g_launches += kernels;
+    return MSA_OK;
+}
+
+// Q [rows, Hq, D] -> box (64, G, 1); K/V [T, Hkv, D] -> box (64, 1, B)
+bool prefill_maps(const Prob &P, const void *q, const void *k, const void *v, CUtensorMap *tq, CUtensorMap *tk,
+                  CUtensorMap *tv) {
+    const uint64_t dq[3] = {(uint64_t)P.D, (uint64_t)P.Hq, (uint64_t)P.T};
+    const uint64_t sq[2] = {(uint64_t)P.D * 2, (uint64_t)P.Hq * P.D * 2};
+    const uint32_t bq[3] = {64, (uint32_t)P.G, 1};
+    const uint64_t dk[3] = {(uint64_t)P.D, (uint64_t)P.Hkv, (uint64_t)P.T};
+    const uint64_t sk[2] = {(uint64_t)P.D * 2, (uint64_t)P.Hkv * P.D * 2};
+    const uint32_t bk[3] = {64, 1, (uint32_t)P.B};
+    return make_map(tq, q, 3, dq, sq, bq) && make_map(tk, k, 3, dk, sk, bk) && make_map(tv, v, 3, dk, sk, bk);
+}
+
+// Q [batch*Hq, D] -> box (64, G); cache [batch*Hkv*Lmax, D] -> box (64, B)
+bool decode_maps(const Prob &P, const void *q, const void *k, const void *v, CUtensorMap *tq, CUtensorMap *tk,
+                 CUtensorMap *tv) {
+    const uint64_t dq[2] = {(uint64_t)P.D, (uint64_t)P.batch * P.Hq};
+    const uint64_t sq[1] = {(uint64_t)P.D * 2};
+    const uint32_t bq[2] = {64, (uint32_t)P.G};
+    const uint64_t dk[2] = {(uint64_t)P.D, (uint64_t)P.batch * P.Hkv * P.Lmax};
+    const uint64_t sk[1] = {(uint64_t)P.D * 2};
+    const uint32_t bk[2] = {64, (uint32_t)P.B};
+    return make_map(tq, q, 2, dq, sq, bq) && make_map(tk, k, 2, dk, sk, bk) && make_map(tv, v, 2, dk, sk, bk);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *msa_status_string(msa_status_t s) {
+    switch (s) {
+        case MSA_OK: return "ok";
+        case MSA_ERR_INVALID_ARG: return "invalid argument";
+        case MSA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MSA_ERR_WORKSPACE: return "workspace too small";
+        case MSA_ERR_CUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+int32_t msa_version(void) { return 100; }
+
+int64_t msa_launch_count(void) { return g_launches.load(); }
+
+msa_status_t msa_index_scores(const msa_config_t *cfg, const msa_shape_t *shape, const void *q, const void *k,
+                              const void *wq, const void *wk, void *k_idx, int64_t kidx_from_block, int64_t row_begin,
+                              int64_t row_end, float *scores, int64_t scores_row_stride, void *q_idx_out,
+                              void *stream) {
+    msa_status_t st = check_cfg(cfg);
+    if (st != MSA_OK) return st;
+    if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
+    if (!q || !wq || !k_idx || !scores || (k && !wk)) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(wq, 16) || !aligned(k_idx, 16) || !aligned(scores, 16) ||
+        (k && (!aligned(k, 16) || !aligned(wk, 16))) || (q_idx_out && !aligned(q_idx_out, 16)))
+        return MSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_end < row_begin || row_end > shape->total_rows || kidx_from_block < 0)
+        return MSA_ERR_INVALID_ARG;
+    if (scores_row_stride < shape->max_blocks || scores_row_stride % 4) return MSA_ERR_INVALID_ARG;
+    const Prob P = make_prob(cfg, shape, row_begin, row_end, nullptr);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int launched = 0;
+    if (k) {
+        cudaError_t e = launch_block_keys(P, k, wk, k_idx, kidx_from_block, s);
+        if (e != cudaSuccess) return MSA_ERR_CUDA;
+        ++launched;
+    }
+    cudaError_t e;
+    if (P.mode == MSA_PREFILL) {
+        if (P.total_blocks == 0 || row_end == row_begin) return cuda_status(cudaSuccess, launched);
+        CUtensorMap tm;
+        const uint64_t dims[3] = {64, (uint64_t)P.Hkv, (uint64_t)P.total_blocks};
+        const uint64_t strides[2] = {128, (uint64_t)P.Hkv * 128};
+        const uint32_t box[3] = {64, 1, 128};
+        if (!make_map(&tm, k_idx, 3, dims, strides, box)) return MSA_ERR_CUDA;
+        e = launch_index_scores_prefill(P, tm, q, wq, scores, scores_row_stride, q_idx_out, s);
+    } else {
+        e = launch_index_scores_decode(P, q, wq, k_idx, scores, scores_row_stride, q_idx_out, s);
+    }
+    return cuda_status(e, launched + (row_end > row_begin ? 1 : 0));
+}
+
+msa_status_t msa_select_topk(const msa_config_t *cfg, const msa_shape_t *shape, const float *scores,
+                             int64_t scores_row_stride, int64_t row_begin, int64_t row_end, int32_t *block_idx,
+                             int32_t *err_flag, void *stream) {
+    msa_status_t st = check_cfg(cfg);
+    if (st != MSA_OK) return st;
+    if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
+    if (!scores || !block_idx || !aligned(scores, 4) || !aligned(block_idx, 4)) return MSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_end < row_begin || row_end > shape->total_rows) return MSA_ERR_INVALID_ARG;
+    if (scores_row_stride < shape->max_blocks) return MSA_ERR_INVALID_ARG;
+    const Prob P = make_prob(cfg, shape, row_begin, row_end, err_flag);
+    cudaError_t e = launch_select_topk(P, scores, scores_row_stride, block_idx, static_cast<cudaStream_t>(stream));
+    return cuda_status(e, row_end > row_begin ? 1 : 0);
+}
+
+msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t *shape, const void *q, const void *k,
+                                     const void *v, const int32_t *block_idx, int64_t row_begin, int64_t row_end,
+                                     void *o, float *lse, void *workspace, size_t *workspace_bytes, int32_t *err_flag,
+                                     void *stream) {
+    msa_status_t st = check_cfg(cfg);
+    if (st != MSA_OK) return st;
+    if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
+    if (shape->mode != MSA_PREFILL || !workspace_bytes) return MSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_end < row_begin || row_end > shape->total_rows) return MSA_ERR_INVALID_ARG;
+    const int64_t R = row_end - row_begin;
+    if (R >= ((int64_t)1 << 23) || R * cfg->num_kv_heads * (cfg->n_topk + 1 + cfg->use_sink) >= ((int64_t)1 << 31))
+        return MSA_ERR_UNSUPPORTED;
+    const Prob P = make_prob(cfg, shape, row_begin, row_end, err_flag);
+    const size_t need = prefill_ws_layout(P, R, nullptr).total;
+    if (!workspace) {
+        *workspace_bytes = need;
+        return MSA_OK;
+    }
+    if (*workspace_bytes < need) return MSA_ERR_WORKSPACE;
+    if (!q || !k || !v || !block_idx || !o) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(block_idx, 4) ||
+        !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+        return MSA_ERR_INVALID_ARG;
+    if (R == 0) return MSA_OK;
+    CUtensorMap tq, tk, tv;
+    if (!prefill_maps(P, q, k, v, &tq, &tk, &tv)) return MSA_ERR_CUDA;
+    cudaError_t e = launch_sparse_prefill(P, tq, tk, tv, block_idx, o, lse, workspace, num_sms(),
+                                          static_cast<cudaStream_t>(stream));
+    return cuda_status(e, 6);
+}
+
+msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *shape, const void *q,
+                                    const void *k_cache, const void *v_cache, const int32_t *block_idx, void *o,
+                                    float *lse, void *workspace, size_t *workspace_bytes, int32_t *err_flag,
+                                    void *stream) {
+    msa_status_t st = check_cfg(cfg);
+    if (st != MSA_OK) return st;
+    if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
+    if (shape->mode != MSA_DECODE || !workspace_bytes) return MSA_ERR_INVALID_ARG;
+    const Prob P = make_prob(cfg, shape, 0, shape->batch, err_flag);
+    int nct, rounds;
+    decode_geometry(P, false, nct, rounds);
+    const size_t need = decode_ws_bytes(P, nct);
+    if (!workspace) {
+        *workspace_bytes = need;
+        return MSA_OK;
+    }
+    if (*workspace_bytes < need) return MSA_ERR_WORKSPACE;
+    if (!q || !k_cache || !v_cache || !block_idx || !o) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+        !aligned(block_idx, 4) || !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+        return MSA_ERR_INVALID_ARG;
+    CUtensorMap tq, tk, tv;
+    if (!decode_maps(P, q, k_cache, v_cache, &tq, &tk, &tv)) return MSA_ERR_CUDA;
+    cudaError_t e = launch_decode(P, tq, tk, tv, block_idx, o, lse, workspace, static_cast<cudaStream_t>(stream));
+    return cuda_status(e, 1);
+}
+
+msa_status_t msa_dense_attn_prefill(const msa_config_t *cfg, const msa_shape_t *shape, const void *q, const void *k,
+                                    const void *v, int64_t row_begin, int64_t row_end, void *o, float *lse,
+                                    int32_t *err_flag, void *stream) {
+    msa_status_t st = check_cfg(cfg);
+    if (st != MSA_OK) return st;
+    if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
+    if (shape->mode != MSA_PREFILL) return MSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_end < row_begin || row_end > shape->total_rows) return MSA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4)))
+        return MSA_ERR_INVALID_ARG;
+    if (row_end == row_begin) return MSA_OK;
+    const Prob P = make_prob(cfg, shape, row_begin, row_end, err_flag);
+    CUtensorMap tq, tk, tv;
+    if (!prefill_maps(P, q, k, v, &tq, &tk, &tv)) return MSA_ERR_CUDA;
+    return cuda_status(launch_dense_prefill(P, tq, tk, tv, o, lse, static_cast<cudaStream_t>(stream)), 1);
+}
+
+msa_status_t msa_dense_attn_decode(const msa_config_t *cfg, const msa_shape_t *shape, const void *q,
+                                   const void *k_cache, const void *v_cache, void *o, float *lse, void *workspace,
+                                   size_t *workspace_bytes, int32_t *err_flag, void *stream) {
+    msa_status_t st = check_cfg(cfg);
+    if (st != MSA_OK) return st;
+    if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
+    if (shape->mode != MSA_DECODE || !workspace_bytes) return MSA_ERR_INVALID_ARG;
+    const Prob P = make_prob(cfg, shape, 0, shape->batch, err_flag);
+    int nct, rounds;
+    decode_geometry(P, true, nct, rounds);
+    const size_t need = decode_ws_bytes(P, nct);
+    if (!workspace) {
+        *workspace_bytes = need;
+        return MSA_OK;
+    }
+    if (*workspace_bytes < need) return MSA_ERR_WORKSPACE;
+    if (!q || !k_cache || !v_cache || !o) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+        !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+        return MSA_ERR_INVALID_ARG;
+    CUtensorMap tq, tk, tv;
+    if (!decode_maps(P, q, k_cache, v_cache, &tq, &tk, &tv)) return MSA_ERR_CUDA;
+    return cuda_status(launch_decode(P, tq, tk, tv, nullptr, o, lse, workspace, static_cast<cudaStream_t>(stream)), 1);
+}
+
+}  // extern "C"

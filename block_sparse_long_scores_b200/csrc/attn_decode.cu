@@ -1,0 +1,349 @@
+// attn_decode.cu -- MSA main branch for decode: one new token per sequence attends exactly to the
+// selected blocks of its KV cache ("深度解析 MiniMax-M3", section "架构核心：MoE 与 MSA 的深度融合",
+// item 2).  Also serves the dense decode baseline (every block 0..i selected).
+//
+// Decode is bound by HBM bandwidth: per (sequence, kv head) it streams k_tot blocks of K and V
+// (16 KB each at D=128, B=64) against only G = 8 query rows.  That is below tcgen05's minimum M of
+// 64, so the contraction uses warp-level mma.sync (m16n8k16, bf16 in, fp32 accumulate) on
+// 128-byte-swizzled tiles that TMA streams in; the tensor pipe is never this kernel's limit.
+//
+// Grid (ctas_per_bg, Hkv, batch).  A CTA has NW warps; in each round every warp takes one block
+// (TMA into its own K/V slot), computes S = Q K^T, an online-softmax update and O += P V.  The
+// warps' states are merged in shared memory into one split partial (m, l, O) per CTA.  The last
+// CTA of a (sequence, kv head) to finish (atomic ticket, no waiting) merges all splits:
+//   m = max_c m_c;  l = sum_c l_c 2^(m_c - m);  O = sum_c O_c 2^(m_c - m) / l;  lse = (m + log2 l) ln 2
+// (scores are kept in log2 units: t = scale * log2(e) * q.k).
+#include "launch.cuh"
+
+namespace msa {
+
+template <int D, int BLK, int NW>
+struct DecSmem {
+    static constexpr int DC = D / 64;
+    static constexpr int KV_CHUNK = BLK * 128;
+    alignas(1024) unsigned char q[DC * 2048];                 // 16 rows x 128 B per chunk
+    alignas(1024) unsigned char k[NW][DC * KV_CHUNK];
+    alignas(1024) unsigned char v[NW][DC * KV_CHUNK];
+    alignas(8) uint64_t bar_q;
+    alignas(8) uint64_t bar[NW];
+    int js[NW];
+    float red_m[NW][16], red_l[NW][16];
+    int fail, last;
+};
+
+struct DecodeBufs {
+    float *ws_m;          // [batch*Hkv, nct, 16]
+    float *ws_l;          // [batch*Hkv, nct, 16]
+    float *ws_o;          // [batch*Hkv, nct, 16, D]
+    int32_t *tickets;     // [batch*Hkv], zero on entry, left zero on exit
+};
+
+template <int D, int BLK, int NW>
+__global__ void __launch_bounds__(NW * 32) decode_attn_kernel(Prob P, const __grid_constant__ CUtensorMap tm_q,
+                                                              const __grid_constant__ CUtensorMap tm_k,
+                                                              const __grid_constant__ CUtensorMap tm_v,
+                                                              const int32_t *__restrict__ block_idx, int rounds,
+                                                              DecodeBufs W, __nv_bfloat16 *__restrict__ O,
+                                                              float *__restrict__ lse) {
+    using SM = DecSmem<D, BLK, NW>;
+    constexpr int DC = SM::DC;
+    extern __shared__ unsigned char smem_raw[];
+    SM &S = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.z, g = blockIdx.y, cta = blockIdx.x, nct = gridDim.x;
+    const int64_t bg = (int64_t)b * P.Hkv + g;
+    const int64_t len = P.seqlens[b];
+    const int64_t pos = len - 1;
+    const int64_t i = pos / BLK;
+    const bool dense = block_idx == nullptr;
+
+    if (tid == 0) {
+        mbar_init(&S.bar_q, 1);
+        for (int w = 0; w < NW; ++w) mbar_init(&S.bar[w], 1);
+        S.fail = 0;
+        fence_barrier_init();
+    }
+    for (int x = tid; x < DC * 2048 / 16; x += NW * 32) reinterpret_cast<uint4 *>(S.q)[x] = make_uint4(0, 0, 0, 0);
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&S.bar_q, P.G * D * 2);
+#pragma unroll
+        for (int c = 0; c < DC; ++c) tma_load_2d(S.q + c * 2048, &tm_q, &S.bar_q, c * 64, b * P.Hq + g * P.G);
+    }
+    bool q_ready = false;
+    bool my_pending = false;     // a load for this warp's slot was issued and not yet seen complete
+    uint32_t my_phase = 0;
+
+    // online-softmax state of this warp: rows r0 = lane/4 and r1 = lane/4 + 8
+    float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
+    float o[D / 8][4];
+#pragma unroll
+    for (int dt = 0; dt < D / 8; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+
+    const uint32_t q_base = smem_u32(S.q);
+    for (int rd = 0; rd < rounds; ++rd) {
+        // which block does this warp take this round?
+        const int64_t a = ((int64_t)cta * rounds + rd) * NW + warp;
+        int j = -1;
+        if (dense) {
+            j = a <= i ? (int)a : -1;
+        } else if (a < P.k_tot) {
+            const int32_t *row = block_idx + bg * P.k_tot;
+            j = row[a];
+            int bad = 0;
+            if (j < -1 || j > i) { bad = kErrBlockRange; j = -1; }
+            if (j >= 0) {
+                bool dup = false;
+                for (int c = lane; c < a; c += 32) dup |= (row[c] == j);
+                if (__any_sync(0xffffffffu, dup)) { bad = kErrDuplicate; j = -1; }
+            }
+            if (bad && lane == 0) report(P.err, bad);
+        }
+        if (lane == 0) S.js[warp] = j;
+        __syncthreads();
+        if (tid == 0) {
+            for (int w = 0; w < NW; ++w) {
+                const int jw = S.js[w];
+                if (jw < 0) continue;
+                const int row0 = (int)(bg * P.Lmax + (int64_t)jw * BLK);
+                mbar_arrive_expect_tx(&S.bar[w], 2 * DC * SM::KV_CHUNK);
+#pragma unroll
+                for (int c = 0; c < DC; ++c) {
+                    tma_load_2d(S.k[w] + c * SM::KV_CHUNK, &tm_k, &S.bar[w], c * 64, row0);
+                    tma_load_2d(S.v[w] + c * SM::KV_CHUNK, &tm_v, &S.bar[w], c * 64, row0);
+                }
+            }
+        }
+        if (j >= 0) {
+            my_pending = true;
+            bool ok = true;
+            if (!q_ready) { ok &= mbar_wait(&S.bar_q, 0); q_ready = true; }
+            const bool landed = mbar_wait(&S.bar[warp], my_phase);
+            if (landed) { my_pending = false; my_phase ^= 1; }
+            ok &= landed;
+            if (!ok && lane == 0) S.fail = 1;
+            const uint32_t k_base = smem_u32(S.k[warp]), v_base = smem_u32(S.v[warp]);
+            // S = Q K^T : 16 rows x BLK keys
+            float s[BLK / 8][4];
+#pragma unroll
+            for (int nt = 0; nt < BLK / 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const int c = ks / 4;
+                uint32_t af[4];
+                {
+                    const int mi = lane >> 3;
+                    const int row = (mi & 1) * 8 + (lane & 7);
+                    const int ch = (ks * 2 + (mi >> 1)) & 7;
+                    ldsm_x4(q_base + c * 2048 + sw128(row, ch), af[0], af[1], af[2], af[3]);
+                }
+#pragma unroll
+                for (int nt = 0; nt < BLK / 8; nt += 2) {
+                    const int mi = lane >> 3;
+                    const int key = (nt + (mi >> 1)) * 8 + (lane & 7);
+                    const int ch = (ks * 2 + (mi & 1)) & 7;
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(k_base + c * SM::KV_CHUNK + sw128(key, ch), b0, b1, b2, b3);
+                    mma_bf16_16816(s[nt], af, b0, b1);
+                    mma_bf16_16816(s[nt + 1], af, b2, b3);
+                }
+            }
+            // scale to log2 units, causal mask on the local block, online-softmax update
+            const int lim = (j == i) ? (int)(pos - (int64_t)j * BLK) : BLK - 1;
+            float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+            for (int nt = 0; nt < BLK / 8; ++nt)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int key = nt * 8 + 2 * (lane & 3) + (x & 1);
+                    const float t = key <= lim ? s[nt][x] * P.scale_log2 : -INFINITY;
+                    s[nt][x] = t;
+                    mx[x >> 1] = fmaxf(mx[x >> 1], t);
+                }
+            float alpha[2];
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
+                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
+                const float m_new = fmaxf(m_r[rr], mx[rr]);
+                alpha[rr] = exp2f(m_r[rr] - m_new);
+                m_r[rr] = m_new;
+            }
+            float ls[2] = {0.f, 0.f};
+#pragma unroll
+            for (int nt = 0; nt < BLK / 8; ++nt)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const float p = exp2f(s[nt][x] - m_r[x >> 1]);
+                    s[nt][x] = p;
+                    ls[x >> 1] += p;
+                }
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) l_r[rr] = l_r[rr] * alpha[rr] + ls[rr];
+#pragma unroll
+            for (int dt = 0; dt < D / 8; ++dt) {
+                o[dt][0] *= alpha[0];
+                o[dt][1] *= alpha[0];
+                o[dt][2] *= alpha[1];
+                o[dt][3] *= alpha[1];
+            }
+            // O += P V
+#pragma unroll
+            for (int kt = 0; kt < BLK / 16; ++kt) {
+                uint32_t pa[4];
+                pa[0] = pack_bf16(s[2 * kt][0], s[2 * kt][1]);
+                pa[1] = pack_bf16(s[2 * kt][2], s[2 * kt][3]);
+                pa[2] = pack_bf16(s[2 * kt + 1][0], s[2 * kt + 1][1]);
+                pa[3] = pack_bf16(s[2 * kt + 1][2], s[2 * kt + 1][3]);
+#pragma unroll
+                for (int dt = 0; dt < D / 8; dt += 2) {
+                    const int mi = lane >> 3;
+                    const int key = kt * 16 + (mi & 1) * 8 + (lane & 7);
+                    const int dch = dt + (mi >> 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(v_base + (dch >> 3) * SM::KV_CHUNK + sw128(key, dch & 7), b0, b1, b2, b3);
+                    mma_bf16_16816(o[dt], pa, b0, b1);
+                    mma_bf16_16816(o[dt + 1], pa, b2, b3);
+                }
+            }
+        }
+        __syncthreads();   // K/V slots are reloaded next round
+        if (S.fail) break;
+    }
+
+    // merge the warps' states into this CTA's split partial
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        l_r[rr] += __shfl_xor_sync(0xffffffffu, l_r[rr], 1);
+        l_r[rr] += __shfl_xor_sync(0xffffffffu, l_r[rr], 2);
+    }
+    if ((lane & 3) == 0) {
+        S.red_m[warp][lane >> 2] = m_r[0];
+        S.red_m[warp][(lane >> 2) + 8] = m_r[1];
+        S.red_l[warp][lane >> 2] = l_r[0];
+        S.red_l[warp][(lane >> 2) + 8] = l_r[1];
+    }
+    float *obuf = reinterpret_cast<float *>(S.k[0]);   // NW x 16 x D fp32 fits in the K slots
+#pragma unroll
+    for (int dt = 0; dt < D / 8; ++dt) {
+        const int col = dt * 8 + 2 * (lane & 3);
+        const int r0 = lane >> 2;
+        obuf[(warp * 16 + r0) * D + col] = o[dt][0];
+        obuf[(warp * 16 + r0) * D + col + 1] = o[dt][1];
+        obuf[(warp * 16 + r0 + 8) * D + col] = o[dt][2];
+        obuf[(warp * 16 + r0 + 8) * D + col + 1] = o[dt][3];
+    }
+    __syncthreads();
+    const int64_t slot = bg * nct + cta;
+    for (int x = tid; x < P.G * D; x += NW * 32) {
+        const int r = x / D, col = x % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, S.red_m[w][r]);
+        float L = 0.f, acc = 0.f;
+        if (M > -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float f = exp2f(S.red_m[w][r] - M);
+                L += S.red_l[w][r] * f;
+                acc += obuf[(w * 16 + r) * D + col] * f;
+            }
+        }
+        W.ws_o[(slot * 16 + r) * D + col] = acc;
+        if (col == 0) {
+            W.ws_m[slot * 16 + r] = M;
+            W.ws_l[slot * 16 + r] = L;
+        }
+    }
+    // last CTA of this (b, g) merges every split
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) S.last = atomicAdd(&W.tickets[bg], 1) == nct - 1;
+    __syncthreads();
+    if (S.last) {
+        __threadfence();
+        for (int x = tid; x < P.G * D; x += NW * 32) {
+            const int r = x / D, col = x % D;
+            float M = -INFINITY;
+            for (int c = 0; c < nct; ++c) M = fmaxf(M, __ldcg(&W.ws_m[(bg * nct + c) * 16 + r]));
+            float L = 0.f, acc = 0.f;
+            if (M > -INFINITY) {
+                for (int c = 0; c < nct; ++c) {
+                    const int64_t sl = bg * nct + c;
+                    const float f = exp2f(__ldcg(&W.ws_m[sl * 16 + r]) - M);
+                    L += __ldcg(&W.ws_l[sl * 16 + r]) * f;
+                    acc += __ldcg(&W.ws_o[(sl * 16 + r) * D + col]) * f;
+                }
+            }
+            const int64_t orow = (int64_t)b * P.Hq + (int64_t)g * P.G + r;
+            O[orow * D + col] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+            if (lse && col == 0) lse[orow] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+        }
+        if (tid == 0) W.tickets[bg] = 0;
+    }
+    if (S.fail) {
+        if (tid == 0) report(P.err, kErrTimeout);
+        // let a copy still in flight into this warp's slot land before the CTA exits
+        if (my_pending && lane == 0) mbar_wait(&S.bar[warp], my_phase);
+    }
+}
+
+// ------------------------------------------------------------------------------ launchers
+
+constexpr int kDecWarps = 2;
+
+size_t decode_ws_bytes(const Prob &P, int nct) {
+    const size_t nbg = (size_t)P.batch * P.Hkv;
+    auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
+    return a(sizeof(float) * nbg * nct * 16) * 2 + a(sizeof(float) * nbg * nct * 16 * P.D) + a(sizeof(int32_t) * nbg);
+}
+
+// Splits per (sequence, kv head) and rounds per CTA.
+void decode_geometry(const Prob &P, bool dense, int &nct, int &rounds) {
+    if (!dense) {
+        rounds = 1;
+        nct = (int)ceil_div<int64_t>(P.k_tot, kDecWarps);
+    } else {
+        const int64_t items = P.max_blocks;
+        rounds = (int)lmax(1, ceil_div<int64_t>(items, (int64_t)kDecWarps * 64));
+        nct = (int)ceil_div<int64_t>(items, (int64_t)kDecWarps * rounds);
+    }
+}
+
+template <int D, int BLK>
+static cudaError_t launch_dec_t(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                const int32_t *block_idx, int nct, int rounds, const DecodeBufs &W, void *O,
+                                float *lse, cudaStream_t st) {
+    const size_t smem = sizeof(DecSmem<D, BLK, kDecWarps>) + 1024;
+    auto kern = decode_attn_kernel<D, BLK, kDecWarps>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)nct, (unsigned)P.Hkv, (unsigned)P.batch);
+    kern<<<grid, kDecWarps * 32, smem, st>>>(P, tq, tk, tv, block_idx, rounds, W, (__nv_bfloat16 *)O, lse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                          const int32_t *block_idx, void *O, float *lse, void *ws, cudaStream_t st) {
+    int nct, rounds;
+    decode_geometry(P, block_idx == nullptr, nct, rounds);
+    const size_t nbg = (size_t)P.batch * P.Hkv;
+    auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
+    char *base = static_cast<char *>(ws);
+    DecodeBufs W;
+    W.ws_m = reinterpret_cast<float *>(base);
+    W.ws_l = reinterpret_cast<float *>(base + a(sizeof(float) * nbg * nct * 16));
+    W.ws_o = reinterpret_cast<float *>(base + 2 * a(sizeof(float) * nbg * nct * 16));
+    W.tickets = reinterpret_cast<int32_t *>(base + 2 * a(sizeof(float) * nbg * nct * 16) +
+                                            a(sizeof(float) * nbg * nct * 16 * P.D));
+    cudaError_t e = cudaMemsetAsync(W.tickets, 0, sizeof(int32_t) * nbg, st);
+    if (e != cudaSuccess) return e;
+    if (P.D == 128 && P.B == 64) return launch_dec_t<128, 64>(P, tq, tk, tv, block_idx, nct, rounds, W, O, lse, st);
+    if (P.D == 128 && P.B == 128) return launch_dec_t<128, 128>(P, tq, tk, tv, block_idx, nct, rounds, W, O, lse, st);
+    if (P.D == 64 && P.B == 64) return launch_dec_t<64, 64>(P, tq, tk, tv, block_idx, nct, rounds, W, O, lse, st);
+    if (P.D == 64 && P.B == 128) return launch_dec_t<64, 128>(P, tq, tk, tv, block_idx, nct, rounds, W, O, lse, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace msa

@@ -1,0 +1,39 @@
+// launch.cuh -- host-side entry points of the kernel translation units, used by abi.cu.
+#pragma once
+
+#include "common.cuh"
+
+namespace msa {
+
+// index.cu
+cudaError_t launch_block_keys(const Prob &P, const void *K, const void *Wk, void *kidx, int64_t from_block,
+                              cudaStream_t st);
+cudaError_t launch_index_scores_prefill(const Prob &P, const CUtensorMap &tm_kidx, const void *Q, const void *Wq,
+                                        float *scores, int64_t stride, void *qidx_out, cudaStream_t st);
+cudaError_t launch_index_scores_decode(const Prob &P, const void *Q, const void *Wq, const void *kidx, float *scores,
+                                       int64_t stride, void *qidx_out, cudaStream_t st);
+// topk.cu
+cudaError_t launch_select_topk(const Prob &P, const float *scores, int64_t stride, int32_t *out, cudaStream_t st);
+
+// attn_prefill.cu
+struct PrefillWs {
+    int32_t *sanitized, *counts, *list_off, *cursor, *entries, *tile_off;
+    int4 *tiles;
+    __nv_bfloat16 *part_o;
+    float *part_lse;
+    size_t total;
+};
+PrefillWs prefill_ws_layout(const Prob &P, int64_t R, void *base);
+cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                  const int32_t *block_idx, void *O, float *lse, void *ws, int num_sms,
+                                  cudaStream_t st);
+// attn_decode.cu
+size_t decode_ws_bytes(const Prob &P, int nct);
+void decode_geometry(const Prob &P, bool dense, int &nct, int &rounds);
+cudaError_t launch_decode(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                          const int32_t *block_idx, void *O, float *lse, void *ws, cudaStream_t st);
+// attn_dense.cu
+cudaError_t launch_dense_prefill(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                 void *O, float *lse, cudaStream_t st);
+
+}  // namespace msa

@@ -1,0 +1,205 @@
+// topk.cu -- MSA index branch, selection step: per-GQA-group top-k over raw logits with no
+// exponential ("exp-free Top-k" of the wiki.500nian.com digest's two-branch flowchart; top-k
+// per GQA group, "深度解析 MiniMax-M3", section "架构核心：MoE 与 MSA 的深度融合", item 1).
+//
+// One CTA per (row, kv head).  The row's candidate scores S[j], j in [use_sink, i), are held in
+// registers as order-preserving uint32 keys (THREADS x E of them, element e of thread t is
+// j = use_sink + t + THREADS * e).  An MSB-first radix select (four 8-bit passes over a shared
+// 256-bin histogram) finds the k-th largest key T and how many keys equal to T are still needed;
+// the picks are every key > T plus the first such keys == T in ascending block order (ties go
+// to the lower block).  Ordered block-wide prefix counts then write the picks in ascending
+// block order, with the sink block in front and the local block behind them.
+#include "launch.cuh"
+
+namespace msa {
+
+template <int THREADS, int E>
+struct TopkSmem {
+    static constexpr int NW = THREADS / 32;
+    unsigned int hist[256];
+    int tot[E * NW];
+    int pre[E * NW];
+    int digit, above, total;
+};
+
+// Exclusive prefix count of `flag` over elements in ascending block order; returns the total.
+template <int THREADS, int E>
+__device__ __forceinline__ int ordered_prefix(const bool (&flag)[E], int (&pos)[E], TopkSmem<THREADS, E> &S) {
+    constexpr int NW = THREADS / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const unsigned bal = __ballot_sync(0xffffffffu, flag[e]);
+        pos[e] = __popc(bal & lt);
+        if (lane == 0) S.tot[e * NW + warp] = __popc(bal);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        constexpr int N = E * NW;
+        constexpr int PER = (N + 31) / 32;
+        int loc[PER];
+        int sum = 0;
+#pragma unroll
+        for (int q = 0; q < PER; ++q) {
+            const int idx = lane * PER + q;
+            loc[q] = idx < N ? S.tot[idx] : 0;
+            sum += loc[q];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int q = 0; q < PER; ++q) {
+            const int idx = lane * PER + q;
+            if (idx < N) S.pre[idx] = run;
+            run += loc[q];
+        }
+        if (lane == 31) S.total = incl;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < E; ++e) pos[e] += S.pre[e * NW + warp];
+    const int total = S.total;
+    __syncthreads();
+    return total;
+}
+
+template <int THREADS, int E>
+__global__ void __launch_bounds__(THREADS) topk_kernel(Prob P, const float *__restrict__ scores, int64_t stride,
+                                                       int32_t *__restrict__ out) {
+    __shared__ TopkSmem<THREADS, E> S;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t rr = blockIdx.x / P.Hkv;
+    const int g = blockIdx.x % P.Hkv;
+    const int64_t row = P.row_begin + rr;
+    const RowGeo geo = row_geo(P, row);
+    const int64_t i = geo.pos / P.B;
+    const int s = P.use_sink;
+    const float *Sr = scores + (rr * P.Hkv + g) * stride;
+    int32_t *o = out + (rr * P.Hkv + g) * (int64_t)P.k_tot;
+
+    // key 0 marks "no candidate" (past the range, or a NaN score); every number maps above 0
+    uint32_t key[E];
+    int n_nan_local = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int64_t j = s + tid + (int64_t)THREADS * e;
+        bool nan = false;
+        key[e] = j < i ? ordered_key(Sr[j], nan) : 0u;
+        n_nan_local += nan;
+    }
+    int nan_total;
+    {
+        int v = n_nan_local;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) S.tot[warp] = v;
+        __syncthreads();
+        nan_total = 0;
+        for (int w = 0; w < THREADS / 32; ++w) nan_total += S.tot[w];
+        __syncthreads();
+    }
+    if (nan_total > 0 && tid == 0) report(P.err, kErrNanScore);
+
+    const int64_t n_cand = i > s ? i - s : 0;
+    const int64_t n_valid = n_cand - nan_total;
+    const int k = P.n_topk;
+    bool sel[E];
+    if (n_valid <= k || k == 0) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) sel[e] = k > 0 && key[e] != 0u;
+    } else {
+        // radix select of the k-th largest key (keys of 0 sit below every candidate and never
+        // reach the k-th place because more than k candidates are valid)
+        uint32_t prefix = 0u, mask = 0u;
+        int remaining = k;
+#pragma unroll 1
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
+            for (int q = tid; q < 256; q += THREADS) S.hist[q] = 0u;
+            __syncthreads();
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                if ((key[e] & mask) == prefix) atomicAdd(&S.hist[(key[e] >> shift) & 255u], 1u);
+            __syncthreads();
+            if (warp == 0) {
+                // lane l scans bins 255-8l .. 248-8l (descending)
+                unsigned c[8];
+                unsigned sum = 0;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    c[q] = S.hist[255 - 8 * lane - q];
+                    sum += c[q];
+                }
+                unsigned incl = sum;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const unsigned v = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += v;
+                }
+                const unsigned excl = incl - sum;
+                if (excl < (unsigned)remaining && (unsigned)remaining <= incl) {
+                    unsigned cum = excl;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (cum + c[q] >= (unsigned)remaining) {
+                            S.digit = 255 - 8 * lane - q;
+                            S.above = (int)cum;
+                            break;
+                        }
+                        cum += c[q];
+                    }
+                }
+            }
+            __syncthreads();
+            remaining -= S.above;
+            prefix |= (uint32_t)S.digit << shift;
+            mask |= 255u << shift;
+            __syncthreads();
+        }
+        const uint32_t T = prefix;
+        int rank[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) sel[e] = key[e] == T;
+        ordered_prefix<THREADS, E>(sel, rank, S);
+#pragma unroll
+        for (int e = 0; e < E; ++e) sel[e] = key[e] > T || (key[e] == T && rank[e] < remaining);
+    }
+    int pos[E];
+    const int n_sel = ordered_prefix<THREADS, E>(sel, pos, S);
+    const int sinkoff = (s && i > 0) ? 1 : 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (sel[e] && sinkoff + pos[e] < P.k_tot - 1) o[sinkoff + pos[e]] = (int32_t)(s + tid + (int64_t)THREADS * e);
+    if (tid == 0) {
+        if (sinkoff) o[0] = 0;
+        o[sinkoff + n_sel] = (int32_t)i;
+    }
+    for (int q = sinkoff + n_sel + 1 + tid; q < P.k_tot; q += THREADS) o[q] = -1;
+}
+
+template <int THREADS, int E>
+static cudaError_t launch_topk_t(const Prob &P, const float *scores, int64_t stride, int32_t *out, cudaStream_t st) {
+    const int64_t n = (P.row_end - P.row_begin) * P.Hkv;
+    topk_kernel<THREADS, E><<<(unsigned)n, THREADS, 0, st>>>(P, scores, stride, out);
+    return cudaGetLastError();
+}
+
+// A row has at most max_blocks - 1 candidates; rows longer than 32768 blocks are refused on the host.
+cudaError_t launch_select_topk(const Prob &P, const float *scores, int64_t stride, int32_t *out, cudaStream_t st) {
+    if (P.row_end <= P.row_begin) return cudaSuccess;
+    const int64_t nmax = P.max_blocks;
+    if (nmax <= 128 * 4) return launch_topk_t<128, 4>(P, scores, stride, out, st);
+    if (nmax <= 128 * 16) return launch_topk_t<128, 16>(P, scores, stride, out, st);
+    if (nmax <= 256 * 32) return launch_topk_t<256, 32>(P, scores, stride, out, st);
+    if (nmax <= 512 * 32) return launch_topk_t<512, 32>(P, scores, stride, out, st);
+    if (nmax <= 1024 * 32) return launch_topk_t<1024, 32>(P, scores, stride, out, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace msa

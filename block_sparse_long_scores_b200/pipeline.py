@@ -1,0 +1,113 @@
+"""The MSA hot path end to end on device tensors: index scores -> top-k -> sparse attention.
+
+This module only allocates buffers (torch) and calls the four C-ABI entry points in order,
+chunking prefill rows so that the score buffer and the attention workspace stay bounded.
+Every arithmetic step runs in the library's kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import msa
+from .workloads import Workload
+
+
+def _ceil4(x: int) -> int:
+    return (x + 3) // 4 * 4
+
+
+class Prefill:
+    """Packed prefill of workload `w` on inputs `x` (device tensors from workloads.make_inputs)."""
+
+    def __init__(self, w: Workload, x: dict, chunk_rows: int | None = None, with_lse: bool = True):
+        assert w.mode == "prefill"
+        self.w, self.x = w, x
+        dev = x["q"].device
+        self.cfg = msa.make_config(w.Hq, w.Hkv, w.D, w.B, w.d, w.n_topk, w.use_sink)
+        self.cu_seqlens = x["cu_seqlens"].to(dev, torch.int32).contiguous()
+        self.cu_blocks = x["cu_blocks"].to(dev, torch.int32).contiguous()
+        self.shape = msa.prefill_shape(self.cu_seqlens, self.cu_blocks, list(w.seqlens), w.B)
+        T, nblk = self.shape.total_rows, self.shape.total_blocks
+        self.stride = _ceil4(self.shape.max_blocks)
+        self.chunk = T if chunk_rows is None else max(1, min(chunk_rows, T))
+        self.given_kidx = "k_idx" in x
+        self.k_idx = x["k_idx"] if self.given_kidx else torch.empty(nblk, w.Hkv, w.d, dtype=torch.bfloat16, device=dev)
+        self.scores = torch.empty(self.chunk, w.Hkv, self.stride, dtype=torch.float32, device=dev)
+        self.block_idx = torch.empty(T, w.Hkv, w.k_tot, dtype=torch.int32, device=dev)
+        self.o = torch.empty(T, w.Hq, w.D, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(T, w.Hq, dtype=torch.float32, device=dev) if with_lse else None
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        ws = msa.msa_sparse_attn_prefill(self.cfg, self.shape, None, None, None, None, 0, self.chunk, None, None, None)
+        self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+
+    def chunks(self):
+        T = self.shape.total_rows
+        for r0 in range(0, T, self.chunk):
+            yield r0, min(T, r0 + self.chunk)
+
+    def index(self, r0: int, r1: int, compute_keys: bool, q_idx_out=None):
+        x = self.x
+        k = None if (self.given_kidx or not compute_keys) else x["k"]
+        msa.msa_index_scores(self.cfg, self.shape, x["q"], k, x["wq"], x["wk"], self.k_idx, 0, r0, r1,
+                             self.scores, self.stride, q_idx_out)
+
+    def select(self, r0: int, r1: int):
+        msa.msa_select_topk(self.cfg, self.shape, self.scores, self.stride, r0, r1, self.block_idx[r0:r1], self.err)
+
+    def attend(self, r0: int, r1: int):
+        x = self.x
+        msa.msa_sparse_attn_prefill(self.cfg, self.shape, x["q"], x["k"], x["v"], self.block_idx[r0:r1], r0, r1,
+                                    self.o, self.lse, self.workspace, self.err)
+
+    def run(self):
+        """One pass of the whole hot path over every row."""
+        first = True
+        for r0, r1 in self.chunks():
+            self.index(r0, r1, compute_keys=first)
+            first = False
+            self.select(r0, r1)
+            self.attend(r0, r1)
+        return self.o, self.lse
+
+
+class Decode:
+    """One decode step of workload `w`: the new token of every sequence against its cache."""
+
+    def __init__(self, w: Workload, x: dict, with_lse: bool = True):
+        assert w.mode == "decode"
+        self.w, self.x = w, x
+        dev = x["q"].device
+        self.cfg = msa.make_config(w.Hq, w.Hkv, w.D, w.B, w.d, w.n_topk, w.use_sink)
+        self.seqlens = x["seqlens"].to(dev, torch.int32).contiguous()
+        Lmax = x["k"].shape[2]
+        self.shape = msa.decode_shape(self.seqlens, w.batch, Lmax, w.B)
+        self.stride = _ceil4(self.shape.max_blocks)
+        self.given_kidx = "k_idx" in x
+        self.k_idx = (x["k_idx"] if self.given_kidx else
+                      torch.empty(w.batch, w.Hkv, self.shape.max_blocks, w.d, dtype=torch.bfloat16, device=dev))
+        self.scores = torch.empty(w.batch, w.Hkv, self.stride, dtype=torch.float32, device=dev)
+        self.block_idx = torch.empty(w.batch, w.Hkv, w.k_tot, dtype=torch.int32, device=dev)
+        self.o = torch.empty(w.batch, w.Hq, w.D, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(w.batch, w.Hq, dtype=torch.float32, device=dev) if with_lse else None
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        ws = msa.msa_sparse_attn_decode(self.cfg, self.shape, None, None, None, None, None, None, None)
+        self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+        self.keys_ready = self.given_kidx
+
+    def prepare_keys(self):
+        """Block keys of the whole cache (kept by the caller between steps)."""
+        x = self.x
+        msa.msa_index_scores(self.cfg, self.shape, x["q"], x["k"], x["wq"], x["wk"], self.k_idx, 0, 0, 0,
+                             self.scores, self.stride)
+        self.keys_ready = True
+
+    def run(self, q_idx_out=None):
+        x = self.x
+        if not self.keys_ready:
+            self.prepare_keys()
+        msa.msa_index_scores(self.cfg, self.shape, x["q"], None, x["wq"], None, self.k_idx, 0, 0, self.w.batch,
+                             self.scores, self.stride, q_idx_out)
+        msa.msa_select_topk(self.cfg, self.shape, self.scores, self.stride, 0, self.w.batch, self.block_idx, self.err)
+        msa.msa_sparse_attn_decode(self.cfg, self.shape, x["q"], x["k"], x["v"], self.block_idx, self.o, self.lse,
+                                   self.workspace, self.err)
+        return self.o, self.lse

@@ -1,0 +1,130 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every function the
+header declares, rejects bad arguments before launching anything, and sizes workspaces."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_long_scores_b200 import msa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(msa.LIB_PATH):
+        from block_sparse_long_scores_b200 import build
+        build.build()
+    return msa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("msa_index_scores", "msa_select_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} declared in msa.h but not exported"
+    assert set(msa.EXPORTED) <= set(declared_functions())
+
+
+def test_status_strings(L):
+    assert L.msa_status_string(0) == b"ok"
+    assert L.msa_status_string(3) == b"workspace too small"
+
+
+def _cfg(**kw):
+    base = dict(Hq=32, Hkv=4, D=128, B=64, d=64, n_topk=64, use_sink=1)
+    base.update(kw)
+    return msa.make_config(base["Hq"], base["Hkv"], base["D"], base["B"], base["d"], base["n_topk"], base["use_sink"])
+
+
+def _prefill_shape(T=131072, B=64, fake_ptr=0x10000):
+    nb = (T + B - 1) // B
+    return msa.Shape(msa.MSA_PREFILL, 1, fake_ptr, fake_ptr, None, T, nb, T, nb)
+
+
+def _ws(L, cfg, shape, r0, r1):
+    n = ctypes.c_size_t(0)
+    rc = L.msa_sparse_attn_prefill(ctypes.byref(cfg), ctypes.byref(shape), None, None, None, None, r0, r1, None,
+                                   None, None, ctypes.byref(n), None, None)
+    return rc, n.value
+
+
+def test_prefill_workspace_query_is_host_only_and_grows_with_rows(L):
+    cfg, shape = _cfg(), _prefill_shape()
+    rc, small = _ws(L, cfg, shape, 0, 1024)
+    assert rc == 0 and small > 0
+    rc, big = _ws(L, cfg, shape, 0, 16384)
+    assert rc == 0 and big > small
+    # partial outputs dominate: rows x Hkv x k_tot x G x D bf16
+    assert big >= 16384 * 4 * 66 * 8 * 128 * 2
+
+
+def test_decode_workspace_query(L):
+    cfg = _cfg()
+    shape = msa.Shape(msa.MSA_DECODE, 32, None, None, 0x10000, 32, 0, 131072, 2048)
+    n = ctypes.c_size_t(0)
+    rc = L.msa_sparse_attn_decode(ctypes.byref(cfg), ctypes.byref(shape), None, None, None, None, None, None, None,
+                                  ctypes.byref(n), None, None)
+    assert rc == 0 and n.value > 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=96), 2), (dict(B=32), 2), (dict(d=32), 2), (dict(Hq=24, Hkv=8), 2),
+    (dict(Hq=30, Hkv=4), 1), (dict(n_topk=-1), 1), (dict(use_sink=2), 1), (dict(n_topk=300), 2),
+])
+def test_bad_config_is_rejected_before_launch(L, kw, code):
+    cfg, shape = _cfg(**kw), _prefill_shape()
+    rc, _ = _ws(L, cfg, shape, 0, 128)
+    assert rc == code
+
+
+def test_bad_shape_and_ranges_are_rejected(L):
+    cfg = _cfg()
+    assert _ws(L, cfg, _prefill_shape(), 10, 5)[0] == 1          # row_end < row_begin
+    assert _ws(L, cfg, _prefill_shape(), 0, 131073)[0] == 1      # past the rows
+    bad = _prefill_shape()
+    bad.max_blocks = 7
+    assert _ws(L, cfg, bad, 0, 10)[0] == 1                       # inconsistent block count
+    bad = _prefill_shape()
+    bad.cu_seqlens = None
+    assert _ws(L, cfg, bad, 0, 10)[0] == 1                       # missing device array
+    n = ctypes.c_size_t(1)
+    rc = L.msa_sparse_attn_prefill(None, ctypes.byref(_prefill_shape()), None, None, None, None, 0, 1, None, None,
+                                   None, ctypes.byref(n), None, None)
+    assert rc == 1                                               # null config
+
+
+def test_workspace_too_small_and_misaligned(L):
+    cfg, shape = _cfg(), _prefill_shape()
+    _, need = _ws(L, cfg, shape, 0, 256)
+    small = ctypes.c_size_t(need - 1)
+    fake = ctypes.c_void_p(0x100000)
+    rc = L.msa_sparse_attn_prefill(ctypes.byref(cfg), ctypes.byref(shape), fake, fake, fake, fake, 0, 256, fake, None,
+                                   fake, ctypes.byref(small), None, None)
+    assert rc == 3
+    ok = ctypes.c_size_t(need)
+    mis = ctypes.c_void_p(0x100008)
+    rc = L.msa_sparse_attn_prefill(ctypes.byref(cfg), ctypes.byref(shape), mis, fake, fake, fake, 0, 256, fake, None,
+                                   fake, ctypes.byref(ok), None, None)
+    assert rc == 1
+
+
+def test_index_scores_rejects_bad_stride(L):
+    cfg, shape = _cfg(), _prefill_shape()
+    fake = ctypes.c_void_p(0x100000)
+    for stride in (2047, 2050):   # below max_blocks / not a multiple of 4
+        rc = L.msa_index_scores(ctypes.byref(cfg), ctypes.byref(shape), fake, fake, fake, fake, fake, 0, 0, 10, fake,
+                                stride, None, None)
+        assert rc == 1

@@ -1,0 +1,267 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same seeded inputs.
+
+Covers every step of the hot path -- block keys, index queries, index scores, per-group top-k,
+sparse prefill and decode attention with their split-softmax combine -- and the dense GQA
+baseline, at sizes spanning many tiles with ragged tails, the degenerate cases (empty ranges,
+rows with no candidates, k >= candidates, forced score ties) and sharp-logit variants.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_long_scores_b200 import msa
+from block_sparse_long_scores_b200.pipeline import Decode, Prefill
+from block_sparse_long_scores_b200.workloads import WORKLOADS, make_inputs, scaled_down
+from oracle import oracle as orc
+from tests.parity_helpers import (check_attention, check_bf16_near, check_scores, cpu, oracle_shape, row_geometry,
+                                  sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _bits(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _prefill_full_check(w, x, chunk_rows=None, rows=None, check_keys=True):
+    """Run the prefill path on the GPU and compare each step with the oracle on `rows`."""
+    pf = Prefill(w, x, chunk_rows=chunk_rows)
+    T = pf.shape.total_rows
+    rows = np.arange(T) if rows is None else rows
+    xc = cpu(x)
+    sh = oracle_shape(w, xc)
+    # GPU: keys + scores per chunk, keeping the scores of the checked rows
+    S_gpu = np.zeros((len(rows), w.Hkv, pf.stride), np.float32)
+    qidx_gpu = torch.empty(pf.chunk, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV)
+    qidx_rows = np.zeros((len(rows), w.Hkv, w.d), np.uint16)
+    first = True
+    for r0, r1 in pf.chunks():
+        pf.index(r0, r1, compute_keys=first, q_idx_out=qidx_gpu)
+        first = False
+        pf.select(r0, r1)
+        pf.attend(r0, r1)
+        sel = (rows >= r0) & (rows < r1)
+        if sel.any():
+            S_gpu[sel] = pf.scores[torch.as_tensor(rows[sel] - r0, device=DEV)].cpu().numpy()
+            qidx_rows[sel] = _bits(qidx_gpu[torch.as_tensor(rows[sel] - r0, device=DEV)])
+    torch.cuda.synchronize()
+    assert int(pf.err.item()) == 0, f"device error flag {int(pf.err.item())}"
+    # index branch
+    if "k_idx" in xc:
+        kidx_ref = _bits(xc["k_idx"])
+        assert np.array_equal(_bits(pf.k_idx), kidx_ref)
+    else:
+        kidx_ref, khat = orc.block_keys(sh, xc["k"], xc["wk"])
+        if check_keys:
+            check_bf16_near(_bits(pf.k_idx), khat, "k_idx")
+        kidx_ref = _bits(pf.k_idx)          # score the GPU's keys to isolate the GEMM
+    qref, qhat = orc.index_query(sh, xc["q"], xc["wq"], rows)
+    check_bf16_near(qidx_rows, qhat, "q_idx")
+    S_ref = orc.index_scores(sh, qidx_rows, kidx_ref, rows, pf.stride)
+    check_scores(w, xc, rows, S_gpu, S_ref)
+    # selection: bit-exact given the GPU's own scores
+    sel_gpu = pf.block_idx.cpu().numpy()[rows]
+    sel_ref = orc.select_topk_f32(sh, S_gpu, rows)
+    assert np.array_equal(sel_gpu, sel_ref), "block selection differs from the oracle on the GPU's scores"
+    # main branch on the GPU's selection
+    O_ref, L_ref = orc.sparse_attn(sh, xc["q"], xc["k"], xc["v"], sel_gpu, rows)
+    O_gpu = pf.o.float().cpu().numpy()[rows]
+    L_gpu = pf.lse.cpu().numpy()[rows]
+    return check_attention(O_gpu, O_ref, L_gpu, L_ref)
+
+
+def test_library_loads_and_reports_version():
+    assert msa.lib().msa_version() >= 100
+
+
+def test_tiny_prefill_parity():
+    w = WORKLOADS["tiny_prefill"]
+    x = make_inputs(w, device=DEV)
+    _prefill_full_check(w, x)
+
+
+@pytest.mark.parametrize("gain", [11.3137, 45.2548])
+def test_tiny_prefill_sharp_logits(gain):
+    # q, k ~ N(0,1) (gain sqrt(128)) and 4x that: exercises the max-subtraction and rescaling
+    w = WORKLOADS["tiny_prefill"]
+    x = make_inputs(w, device=DEV, logit_gain=gain, seed=1)
+    _prefill_full_check(w, x)
+
+
+def test_prefill_128k_shape_small_multichunk():
+    # the 128K workload's heads/blocks/selection at 6000 rows (ragged tail), three chunks
+    w = scaled_down(WORKLOADS["prefill_128k"], (6000,))
+    x = make_inputs(w, device=DEV, seed=2)
+    _prefill_full_check(w, x, chunk_rows=2048)
+
+
+def test_ragged_prefill_small_with_ties():
+    # ragged workload shape (64/8 heads, D 64, B 128, k 32, discrete index keys -> exact ties)
+    w = scaled_down(WORKLOADS["ragged_prefill"], (1, 130, 1000, 64, 2900, 129, 700))
+    x = make_inputs(w, device=DEV, seed=3)
+    _prefill_full_check(w, x, chunk_rows=1500)
+
+
+def test_prefill_k_covers_all_candidates_equals_dense():
+    # n_topk >= every candidate: the sparse path must reproduce dense causal attention
+    w = scaled_down(WORKLOADS["tiny_prefill"], (700, 1100)).with_(n_topk=40)
+    x = make_inputs(w, device=DEV, seed=4)
+    pf = Prefill(w, x)
+    pf.run()
+    od = torch.empty_like(pf.o)
+    ld = torch.empty_like(pf.lse)
+    msa.msa_dense_attn_prefill(pf.cfg, pf.shape, x["q"], x["k"], x["v"], 0, pf.shape.total_rows, od, ld)
+    torch.cuda.synchronize()
+    xc = cpu(x)
+    sh = oracle_shape(w, xc)
+    rows = np.arange(pf.shape.total_rows)
+    O_ref, L_ref = orc.dense_attn(sh, xc["q"], xc["k"], xc["v"], rows)
+    check_attention(pf.o.float().cpu().numpy(), O_ref, pf.lse.cpu().numpy(), L_ref)
+    check_attention(od.float().cpu().numpy(), O_ref, ld.cpu().numpy(), L_ref)
+
+
+def test_prefill_sink_and_zero_topk():
+    for k, sink in [(0, 0), (0, 1), (3, 1)]:
+        w = scaled_down(WORKLOADS["tiny_prefill"], (300, 5, 64)).with_(n_topk=k, use_sink=sink)
+        x = make_inputs(w, device=DEV, seed=5 + k + sink)
+        _prefill_full_check(w, x)
+
+
+def test_empty_row_range_is_a_no_op():
+    w = WORKLOADS["tiny_prefill"]
+    x = make_inputs(w, device=DEV)
+    pf = Prefill(w, x)
+    pf.o.zero_()
+    before = pf.o.clone()
+    msa.msa_sparse_attn_prefill(pf.cfg, pf.shape, x["q"], x["k"], x["v"], pf.block_idx, 5, 5, pf.o, pf.lse,
+                                pf.workspace)
+    msa.msa_select_topk(pf.cfg, pf.shape, pf.scores, pf.stride, 7, 7, pf.block_idx)
+    torch.cuda.synchronize()
+    assert torch.equal(before, pf.o)
+
+
+def test_bad_block_ids_are_flagged_and_skipped():
+    w = scaled_down(WORKLOADS["tiny_prefill"], (512,))
+    x = make_inputs(w, device=DEV, seed=6)
+    pf = Prefill(w, x)
+    T = pf.shape.total_rows
+    rows = np.arange(T)
+    _, i = row_geometry(w, cpu(x), rows)
+    rng = np.random.default_rng(0)
+    bi = np.full((T, w.Hkv, w.k_tot), -1, np.int32)
+    for r in range(T):
+        for g in range(w.Hkv):
+            pick = sorted(set(rng.integers(0, i[r] + 1, size=3).tolist()) | {int(i[r])})
+            bi[r, g, :len(pick)] = pick
+    clean = bi.copy()
+    bad = bi.copy()
+    bad[10, 0, -1] = 9999            # beyond the local block -> skipped, flagged
+    bad[300, 1, -1] = bad[300, 1, 0]  # repeated block -> skipped, flagged
+    bad[400, 0, 5] = -7              # negative other than -1 -> skipped, flagged
+    dev_bi = torch.as_tensor(bad, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    msa.msa_sparse_attn_prefill(pf.cfg, pf.shape, x["q"], x["k"], x["v"], dev_bi, 0, T, pf.o, pf.lse, pf.workspace, err)
+    torch.cuda.synchronize()
+    flags = int(err.item())
+    assert flags & 1 and flags & 2, flags
+    xc = cpu(x)
+    sh = oracle_shape(w, xc)
+    clean[400, 0, 5] = -1
+    O_ref, L_ref = orc.sparse_attn(sh, xc["q"], xc["k"], xc["v"], clean, rows)
+    check_attention(pf.o.float().cpu().numpy(), O_ref, pf.lse.cpu().numpy(), L_ref)
+
+
+def test_block_order_does_not_matter():
+    w = scaled_down(WORKLOADS["tiny_prefill"], (900,))
+    x = make_inputs(w, device=DEV, seed=7)
+    pf = Prefill(w, x)
+    pf.run()
+    o1 = pf.o.clone()
+    shuffled = pf.block_idx.flip(-1).contiguous()
+    msa.msa_sparse_attn_prefill(pf.cfg, pf.shape, x["q"], x["k"], x["v"], shuffled, 0, pf.shape.total_rows, pf.o,
+                                pf.lse, pf.workspace, pf.err)
+    torch.cuda.synchronize()
+    # the combine sums partials in slot order, so fp32 rounding may differ: same tolerance as parity
+    from tests.parity_helpers import check_attention
+    check_attention(pf.o.float().cpu().numpy(), o1.double().cpu().numpy())
+    assert int(pf.err.item()) == 0
+
+
+# --------------------------------------------------------------------------------- decode
+
+
+def _decode_check(w, x):
+    dc = Decode(w, x)
+    qidx = torch.empty(w.batch, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV)
+    dc.run(q_idx_out=qidx)
+    torch.cuda.synchronize()
+    assert int(dc.err.item()) == 0
+    xc = cpu(x)
+    sh = oracle_shape(w, xc)
+    rows = np.arange(w.batch)
+    if "k_idx" in xc:
+        kidx = _bits(xc["k_idx"])
+    else:
+        kidx_ref, khat = orc.block_keys(sh, xc["k"], xc["wk"])
+        _, i = row_geometry(w, xc, rows)
+        # complete blocks only are ever scored; compare those
+        mask = np.zeros(khat.shape[:3], bool)
+        for b in range(w.batch):
+            mask[b, :, : i[b]] = True
+        check_bf16_near(_bits(dc.k_idx)[mask], khat[mask], "k_idx (cache)")
+        kidx = _bits(dc.k_idx)
+    check_bf16_near(_bits(qidx), orc.index_query(sh, xc["q"], xc["wq"], rows)[1], "q_idx")
+    S_gpu = dc.scores.cpu().numpy()
+    S_ref = orc.index_scores(sh, _bits(qidx), kidx, rows, dc.stride)
+    check_scores(w, xc, rows, S_gpu, S_ref)
+    sel = dc.block_idx.cpu().numpy()
+    assert np.array_equal(sel, orc.select_topk_f32(sh, S_gpu, rows))
+    O_ref, L_ref = orc.sparse_attn(sh, xc["q"], xc["k"], xc["v"], sel, rows)
+    check_attention(dc.o.float().cpu().numpy(), O_ref, dc.lse.cpu().numpy(), L_ref)
+    return dc
+
+
+def test_decode_small_ragged():
+    w = scaled_down(WORKLOADS["decode_128k"], (1, 63, 64, 65, 1000, 4096, 2000, 3333))
+    x = make_inputs(w, device=DEV, seed=8)
+    _decode_check(w, x)
+
+
+def test_decode_ragged_shape_with_ties():
+    w = scaled_down(WORKLOADS["ragged_decode"], (129, 5000, 1, 3000))
+    x = make_inputs(w, device=DEV, seed=9)
+    _decode_check(w, x)
+
+
+def test_dense_decode_matches_oracle():
+    w = scaled_down(WORKLOADS["decode_128k"], (1, 100, 4096, 2500))
+    x = make_inputs(w, device=DEV, seed=10)
+    dc = Decode(w, x)
+    ws = msa.msa_dense_attn_decode(dc.cfg, dc.shape, None, None, None, None, None, None)
+    wsb = torch.empty(max(ws, 256), dtype=torch.uint8, device=DEV)
+    msa.msa_dense_attn_decode(dc.cfg, dc.shape, x["q"], x["k"], x["v"], dc.o, dc.lse, wsb)
+    torch.cuda.synchronize()
+    xc = cpu(x)
+    sh = oracle_shape(w, xc)
+    O_ref, L_ref = orc.dense_attn(sh, xc["q"], xc["k"], xc["v"], np.arange(w.batch))
+    check_attention(dc.o.float().cpu().numpy(), O_ref, dc.lse.cpu().numpy(), L_ref)
+
+
+# ----------------------------------------------------------------- full-size, sampled rows
+
+
+@pytest.mark.slow
+def test_prefill_128k_full_size_sampled():
+    w = WORKLOADS["prefill_128k"]
+    x = make_inputs(w, device=DEV)
+    rows = sample_rows(w, 256)
+    _prefill_full_check(w, x, chunk_rows=16384, rows=rows, check_keys=True)
+
+
+@pytest.mark.slow
+def test_decode_128k_full_size():
+    w = WORKLOADS["decode_128k"]
+    x = make_inputs(w, device=DEV)
+    _decode_check(w, x)
