@@ -5,6 +5,8 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "launch.cuh"
 #include "msa.h"
@@ -15,6 +17,29 @@ using namespace msa;
 namespace {
 
 std::atomic<int64_t> g_launches{0};
+
+// ------------------------------------------------------------------ opt-in per-kernel timing
+
+struct ProfRec {
+    std::string family;
+    cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::atomic<bool> g_prof_on{false};
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_prof_pool;
+thread_local cudaEvent_t t_prof_open = nullptr;
+
+cudaEvent_t prof_event() {
+    if (!g_prof_pool.empty()) {
+        cudaEvent_t e = g_prof_pool.back();
+        g_prof_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
 
 // ------------------------------------------------------------------ driver entry point (TMA)
 
@@ -161,7 +186,54 @@ bool decode_maps(const Prob &P, const void *q, const void *k, const void *v, CUt
 
 }  // namespace
 
+namespace msa {
+void prof_begin(const char *, cudaStream_t st) {
+    if (!g_prof_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    t_prof_open = prof_event();
+    if (t_prof_open) cudaEventRecord(t_prof_open, st);
+}
+void prof_end(const char *family, cudaStream_t st) {
+    if (!g_prof_on.load(std::memory_order_relaxed) || !t_prof_open) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    cudaEvent_t b = prof_event();
+    if (b) {
+        cudaEventRecord(b, st);
+        g_prof_recs.push_back({family, t_prof_open, b});
+    }
+    t_prof_open = nullptr;
+}
+}  // namespace msa
+
 extern "C" {
+
+void msa_profile_enable(int on) { g_prof_on.store(on != 0); }
+
+void msa_profile_reset(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (auto &r : g_prof_recs) {
+        g_prof_pool.push_back(r.a);
+        g_prof_pool.push_back(r.b);
+    }
+    g_prof_recs.clear();
+}
+
+int32_t msa_profile_read(const char *family, double *total_ms, int64_t *launches) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    double ms = 0.0;
+    int64_t n = 0;
+    for (auto &r : g_prof_recs) {
+        if (family && r.family != family) continue;
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+            return MSA_ERR_CUDA;
+        ms += t;
+        ++n;
+    }
+    if (total_ms) *total_ms = ms;
+    if (launches) *launches = n;
+    return MSA_OK;
+}
 
 const char *msa_status_string(msa_status_t s) {
     switch (s) {

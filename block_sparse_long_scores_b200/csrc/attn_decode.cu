@@ -339,6 +339,7 @@ cudaError_t launch_decode(const Prob &P, const CUtensorMap &tq, const CUtensorMa
                                             a(sizeof(float) * nbg * nct * 16 * P.D));
     cudaError_t e = cudaMemsetAsync(W.tickets, 0, sizeof(int32_t) * nbg, st);
     if (e != cudaSuccess) return e;
+    ProfScope prof(block_idx ? "decode_attn" : "dense_decode", st);
     if (P.D == 128 && P.B == 64) return launch_dec_t<128, 64>(P, tq, tk, tv, block_idx, nct, rounds, W, O, lse, st);
     if (P.D == 128 && P.B == 128) return launch_dec_t<128, 128>(P, tq, tk, tv, block_idx, nct, rounds, W, O, lse, st);
     if (P.D == 64 && P.B == 64) return launch_dec_t<64, 64>(P, tq, tk, tv, block_idx, nct, rounds, W, O, lse, st);

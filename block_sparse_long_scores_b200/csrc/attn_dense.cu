@@ -263,6 +263,7 @@ static cudaError_t launch_dense_t(const Prob &P, const CUtensorMap &tq, const CU
 
 cudaError_t launch_dense_prefill(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                  void *O, float *lse, cudaStream_t st) {
+    ProfScope prof("dense_prefill", st);
     cudaError_t e = cudaSuccess;
     if (P.D == 128 && P.B == 64) { MSA_DISPATCH_G2(P.G, e = launch_dense_t<128, 64, G_>(P, tq, tk, tv, O, lse, st)); }
     else if (P.D == 128 && P.B == 128) { MSA_DISPATCH_G2(P.G, e = launch_dense_t<128, 128, G_>(P, tq, tk, tv, O, lse, st)); }

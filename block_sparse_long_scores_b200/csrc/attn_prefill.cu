@@ -516,6 +516,8 @@ cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CU
     const int tpt = 128 / rpt;
     const int64_t L = (int64_t)P.Hkv * P.total_blocks;
     cudaError_t e;
+    {
+    ProfScope prof("prefill_lists", st);
     if ((e = cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * L, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(w.cursor, 0, sizeof(int32_t) * L, st)) != cudaSuccess) return e;
     const int64_t warps = R * P.Hkv;
@@ -531,13 +533,18 @@ cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CU
     prefill_tiles_kernel<<<(unsigned)ceil_div<int64_t>(L, 256), 256, 0, st>>>(L, tpt, w.counts, w.list_off,
                                                                              w.tile_off, w.tiles);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     PrefillBufs W{w.entries, w.tiles, w.tile_off + L, w.part_o, w.part_lse};
+    {
+    ProfScope prof("prefill_attn", st);
     if (P.D == 128 && P.B == 64) { MSA_DISPATCH_G(P.G, e = launch_attn_t<128, 64, G_>(P, tq, tk, tv, W, num_sms, st)); }
     else if (P.D == 128 && P.B == 128) { MSA_DISPATCH_G(P.G, e = launch_attn_t<128, 128, G_>(P, tq, tk, tv, W, num_sms, st)); }
     else if (P.D == 64 && P.B == 64) { MSA_DISPATCH_G(P.G, e = launch_attn_t<64, 64, G_>(P, tq, tk, tv, W, num_sms, st)); }
     else if (P.D == 64 && P.B == 128) { MSA_DISPATCH_G(P.G, e = launch_attn_t<64, 128, G_>(P, tq, tk, tv, W, num_sms, st)); }
     else return cudaErrorInvalidValue;
+    }
     if (e != cudaSuccess) return e;
+    ProfScope prof("prefill_combine", st);
     if (P.D == 128) { MSA_DISPATCH_G(P.G, e = launch_combine_t<128, G_>(P, w, O, lse, st)); }
     else { MSA_DISPATCH_G(P.G, e = launch_combine_t<64, G_>(P, w, O, lse, st)); }
     return e;

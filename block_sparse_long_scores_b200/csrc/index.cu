@@ -333,6 +333,7 @@ cudaError_t launch_block_keys(const Prob &P, const void *K, const void *Wk, void
         cudaError_t e = cudaFuncSetAttribute(block_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
+    ProfScope prof("block_keys", st);
     block_keys_kernel<<<(unsigned)nctas, 256, smem, st>>>(P, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)Wk,
                                                          (__nv_bfloat16 *)kidx, from_block);
     return cudaGetLastError();
@@ -346,6 +347,7 @@ cudaError_t launch_index_scores_prefill(const Prob &P, const CUtensorMap &tm_kid
     if (rows <= 0) return cudaSuccess;
     dim3 grid((unsigned)ceil_div<int64_t>(rows, kIdxRows), (unsigned)P.Hkv);
     const size_t smem = index_tc_smem();
+    ProfScope prof("index_scores", st);
     cudaError_t e;
     if (P.D == 128) {
         e = cudaFuncSetAttribute(index_scores_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -368,6 +370,7 @@ cudaError_t launch_index_scores_decode(const Prob &P, const void *Q, const void 
     const int64_t rows = P.row_end - P.row_begin;
     if (rows <= 0) return cudaSuccess;
     dim3 grid((unsigned)ceil_div<int64_t>(P.max_blocks, 256), (unsigned)P.Hkv, (unsigned)rows);
+    ProfScope prof("index_scores", st);
     if (P.D == 128)
         index_scores_decode_kernel<128><<<grid, 256, 0, st>>>(P, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)Wq,
                                                               (const __nv_bfloat16 *)kidx, scores, stride,

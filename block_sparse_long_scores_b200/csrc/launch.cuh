@@ -5,6 +5,18 @@
 
 namespace msa {
 
+// Opt-in per-kernel timing (abi.cu): when enabled, a launcher wraps each kernel family in a pair
+// of CUDA events on its stream; totals are read back by msa_profile_read.
+void prof_begin(const char *family, cudaStream_t st);
+void prof_end(const char *family, cudaStream_t st);
+
+struct ProfScope {
+    const char *family;
+    cudaStream_t st;
+    ProfScope(const char *f, cudaStream_t s) : family(f), st(s) { prof_begin(family, st); }
+    ~ProfScope() { prof_end(family, st); }
+};
+
 // index.cu
 cudaError_t launch_block_keys(const Prob &P, const void *K, const void *Wk, void *kidx, int64_t from_block,
                               cudaStream_t st);

@@ -193,6 +193,7 @@ static cudaError_t launch_topk_t(const Prob &P, const float *scores, int64_t str
 // A row has at most max_blocks - 1 candidates; rows longer than 32768 blocks are refused on the host.
 cudaError_t launch_select_topk(const Prob &P, const float *scores, int64_t stride, int32_t *out, cudaStream_t st) {
     if (P.row_end <= P.row_begin) return cudaSuccess;
+    ProfScope prof("select_topk", st);
     const int64_t nmax = P.max_blocks;
     if (nmax <= 128 * 4) return launch_topk_t<128, 4>(P, scores, stride, out, st);
     if (nmax <= 128 * 16) return launch_topk_t<128, 16>(P, scores, stride, out, st);

@@ -27,7 +27,7 @@ DERR = {1: "BLOCK_RANGE", 2: "DUPLICATE", 4: "NAN_SCORE", 8: "TIMEOUT", 16: "SHA
 
 EXPORTED = ("msa_index_scores", "msa_select_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
             "msa_dense_attn_prefill", "msa_dense_attn_decode", "msa_status_string", "msa_version",
-            "msa_launch_count")
+            "msa_launch_count", "msa_profile_enable", "msa_profile_reset", "msa_profile_read")
 
 
 class MSAError(RuntimeError):
@@ -84,6 +84,12 @@ def lib() -> ctypes.CDLL:
         L.msa_status_string.restype = ctypes.c_char_p
         L.msa_version.restype = I32
         L.msa_launch_count.restype = I64
+        L.msa_profile_enable.argtypes = [ctypes.c_int]
+        L.msa_profile_enable.restype = None
+        L.msa_profile_reset.argtypes = []
+        L.msa_profile_reset.restype = None
+        L.msa_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64)]
+        L.msa_profile_read.restype = I32
         _lib = L
     return _lib
 
@@ -195,6 +201,22 @@ def msa_dense_attn_decode(cfg: Config, shape: Shape, q, k_cache, v_cache, o, lse
 
 def launch_count() -> int:
     return int(lib().msa_launch_count())
+
+
+def profile_enable(on: bool = True):
+    lib().msa_profile_enable(1 if on else 0)
+
+
+def profile_reset():
+    lib().msa_profile_reset()
+
+
+def profile_read(family: str | None = None):
+    """(total milliseconds, launches) of one kernel family since the last reset."""
+    ms, n = ctypes.c_double(0.0), ctypes.c_int64(0)
+    rc = lib().msa_profile_read(family.encode() if family else None, ctypes.byref(ms), ctypes.byref(n))
+    _check("msa_profile_read", rc)
+    return ms.value, n.value
 
 
 def default_scale(D: int) -> float:

@@ -213,6 +213,18 @@ int32_t msa_version(void);            /* major * 10000 + minor * 100 + patch */
 /* Kernel launches the library made since load (all calls, all devices): for launch accounting. */
 int64_t msa_launch_count(void);
 
+/*
+ * Opt-in per-kernel timing for measurement tools.  While enabled, every kernel family the
+ * library launches (block_keys, index_scores, select_topk, prefill_lists, prefill_attn,
+ * prefill_combine, decode_attn, dense_decode, dense_prefill) is bracketed by a pair of CUDA events
+ * recorded on the caller's stream.  msa_profile_read waits for the recorded events and returns the
+ * summed milliseconds and the number of bracketed launches of one family (NULL: all families);
+ * msa_profile_reset forgets them.  Disabled by default; costs two event records per launch.
+ */
+void msa_profile_enable(int on);
+void msa_profile_reset(void);
+int32_t msa_profile_read(const char *family, double *total_ms, int64_t *launches);
+
 #ifdef __cplusplus
 }
 #endif
