@@ -184,6 +184,28 @@ bool decode_maps(const Prob &P, const void *q, const void *k, const void *v, CUt
     return make_map(tq, q, 2, dq, sq, bq) && make_map(tk, k, 2, dk, sk, bk) && make_map(tv, v, 2, dk, sk, bk);
 }
 
+// Scratch of msa_sparse_attn_decode_noalloc: a fixed array in device global memory, so the
+// call itself never allocates.  Every device that loads this library holds it until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(40) << 20;   // 40 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+// Device address of g_decode_scratch on the current device.  In host code the array's name is
+// only a host-side stand-in, so the address is looked up once per device (with that device
+// current) and cached; nullptr if the lookup fails.
+void *decode_scratch_address() {
+    static std::mutex mu;
+    static void *addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
 }  // namespace
 
 namespace msa {
@@ -400,6 +422,30 @@ msa_status_t msa_dense_attn_decode(const msa_config_t *cfg, const msa_shape_t *s
     CUtensorMap tq, tk, tv;
     if (!decode_maps(P, q, k_cache, v_cache, &tq, &tk, &tv)) return MSA_ERR_CUDA;
     return cuda_status(launch_decode(P, tq, tk, tv, nullptr, o, lse, workspace, static_cast<cudaStream_t>(stream)), 1);
+}
+
+msa_status_t msa_sparse_attn_decode_noalloc(const msa_config_t *cfg, const msa_shape_t *shape, const void *q,
+                                            const void *k_cache, const void *v_cache, const int32_t *block_idx,
+                                            void *o, float *lse, int32_t *err_flag, void *stream) {
+    msa_status_t st = check_cfg(cfg);
+    if (st != MSA_OK) return st;
+    if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
+    if (shape->mode != MSA_DECODE) return MSA_ERR_INVALID_ARG;
+    const Prob P = make_prob(cfg, shape, 0, shape->batch, err_flag);
+    int nct, rounds;
+    decode_geometry(P, false, nct, rounds);
+    if (decode_ws_bytes(P, nct) > kNoAllocScratchBytes) return MSA_ERR_WORKSPACE;   // beyond the fixed scratch
+    if (!q || !k_cache || !v_cache || !block_idx || !o) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+        !aligned(block_idx, 4) || (lse && !aligned(lse, 4)))
+        return MSA_ERR_INVALID_ARG;
+    void *scratch = decode_scratch_address();
+    if (!scratch) return MSA_ERR_CUDA;
+    CUtensorMap tq, tk, tv;
+    if (!decode_maps(P, q, k_cache, v_cache, &tq, &tk, &tv)) return MSA_ERR_CUDA;
+    // launch_decode clears the split tickets in the scratch before its kernel runs
+    cudaError_t e = launch_decode(P, tq, tk, tv, block_idx, o, lse, scratch, static_cast<cudaStream_t>(stream));
+    return cuda_status(e, 1);
 }
 
 }  // extern "C"

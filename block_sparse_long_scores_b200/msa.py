@@ -27,7 +27,8 @@ DERR = {1: "BLOCK_RANGE", 2: "DUPLICATE", 4: "NAN_SCORE", 8: "TIMEOUT", 16: "SHA
 
 EXPORTED = ("msa_index_scores", "msa_select_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
             "msa_dense_attn_prefill", "msa_dense_attn_decode", "msa_status_string", "msa_version",
-            "msa_launch_count", "msa_profile_enable", "msa_profile_reset", "msa_profile_read")
+            "msa_launch_count", "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
+            "msa_sparse_attn_decode_noalloc")
 
 
 class MSAError(RuntimeError):
@@ -75,6 +76,7 @@ def lib() -> ctypes.CDLL:
             "msa_sparse_attn_decode": [CP, SP, P, P, P, P, P, P, P, SZ, P, P],
             "msa_dense_attn_prefill": [CP, SP, P, P, P, I64, I64, P, P, P, P],
             "msa_dense_attn_decode": [CP, SP, P, P, P, P, P, P, SZ, P, P],
+            "msa_sparse_attn_decode_noalloc": [CP, SP, P, P, P, P, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -180,6 +182,17 @@ def msa_sparse_attn_decode(cfg: Config, shape: Shape, q, k_cache, v_cache, block
                                       ctypes.byref(nbytes), _ptr(err_flag), _stream(stream))
     _check("msa_sparse_attn_decode", rc)
     return nbytes.value
+
+
+def msa_sparse_attn_decode_noalloc(cfg: Config, shape: Shape, q, k_cache, v_cache, block_idx, o, lse,
+                                   err_flag=None, stream=None):
+    """msa_sparse_attn_decode without a workspace argument, for callers that cannot allocate:
+    scratch comes from the library's fixed 40 MiB device array (see include/msa.h for the limit,
+    the first-call set-up and why overlapping calls must be serialised)."""
+    rc = lib().msa_sparse_attn_decode_noalloc(ctypes.byref(cfg), ctypes.byref(shape), _ptr(q), _ptr(k_cache),
+                                              _ptr(v_cache), _ptr(block_idx), _ptr(o), _ptr(lse), _ptr(err_flag),
+                                              _stream(stream))
+    _check("msa_sparse_attn_decode_noalloc", rc)
 
 
 def msa_dense_attn_prefill(cfg: Config, shape: Shape, q, k, v, row_begin: int, row_end: int, o, lse,

@@ -192,6 +192,31 @@ msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *
                                     int32_t *err_flag, void *stream);
 
 /*
+ * msa_sparse_attn_decode_noalloc -- msa_sparse_attn_decode for callers that cannot allocate.
+ * The pages have no counterpart; this is a deployment convenience of this library.
+ *
+ * Some callers cannot hand the library a workspace: a host runtime whose device memory is wholly
+ * owned by another allocator, or a serving loop that must not call the CUDA allocator in its
+ * step (cudaMalloc/cudaFree can synchronise the device).  This entry point computes exactly what
+ * msa_sparse_attn_decode computes (same arguments minus the workspace) and takes its scratch from
+ * a fixed 40 MiB array in device global memory that the library declares; it calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *  - Limit: a problem whose split partials need more than 40 MiB (batch x Hkv x
+ *    ceil(k_tot/2) x 16 x (head_dim + 2) x 4 bytes, roughly) returns MSA_ERR_WORKSPACE and
+ *    launches nothing.  The two decode workloads of this repository fit (128K: 35 MiB; 1M: 17 MiB).
+ *  - Set-up: the first call on a device looks up the array's device address (with that device
+ *    current) and caches it; make that first call before any CUDA stream capture.
+ *  - Sharing: every call on a device uses the same array, and the array keeps the last call's
+ *    contents (the call clears what must start at zero itself).  Calls that may overlap on the GPU
+ *    -- on different streams, or from different threads -- race on it: serialise them.
+ *  - Every GPU that loads the library holds the 40 MiB until the process exits.
+ */
+msa_status_t msa_sparse_attn_decode_noalloc(const msa_config_t *cfg, const msa_shape_t *shape,
+                                            const void *q, const void *k_cache, const void *v_cache,
+                                            const int32_t *block_idx, void *o, float *lse,
+                                            int32_t *err_flag, void *stream);
+
+/*
  * Dense causal GQA attention: the speed-up baseline (the "GQA baseline" the digest compares MSA
  * with), not part of the MSA contract.  Same layouts as the sparse calls; every key t <= the row's
  * position in its own sequence is attended.
