@@ -349,7 +349,7 @@ msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t 
     if (R == 0) return MSA_OK;
     CUtensorMap tq, tk, tv;
     if (!prefill_maps(P, q, k, v, &tq, &tk, &tv)) return MSA_ERR_CUDA;
-    cudaError_t e = launch_sparse_prefill(P, tq, tk, tv, block_idx, o, lse, workspace, num_sms(),
+    cudaError_t e = launch_sparse_prefill(P, tq, tk, tv, q, block_idx, o, lse, workspace, num_sms(),
                                           static_cast<cudaStream_t>(stream));
     return cuda_status(e, 6);
 }

@@ -160,6 +160,15 @@ __global__ void prefill_tiles_kernel(int64_t L, int tpt, const int32_t *__restri
 }
 
 // ------------------------------------------------------------------------- tcgen05 attention
+//
+// Warp-specialised persistent kernel; each CTA walks a contiguous range of tiles (tiles of one
+// list are adjacent, so a KV block is loaded once per CTA and list).  Roles:
+//   warp 0      producer: tile contexts, Q gathers (3-stage ring), K/V blocks (2 stages) by TMA
+//   warp 1      MMA issuer: S = Q K^T into one of 2 TMEM S buffers, O = P V into one of 2 TMEM O
+//               buffers; MMA1 of tile t+1 is issued before MMA2 of tile t
+//   warps 4-7   softmax: S (TMEM) -> row max/sum -> bf16 P tile (smem), one thread per row
+//   warps 8-11  epilogue: O (TMEM) -> normalised bf16 partial + lse -> global
+// Hand-offs are mbarriers; "empty" barriers start free (first wait on parity 1 passes).
 
 template <int D, int BLK, int G>
 struct AttnShape {
@@ -168,27 +177,48 @@ struct AttnShape {
     static constexpr int DC = D / 64;             // 64-element chunks of a head vector
     static constexpr int BC = BLK / 64;           // 64-key chunks of a block
     static constexpr int Q_CHUNK = 128 * 128;     // 128 rows x 128 B
+    static constexpr int Q_STAGE = DC * Q_CHUNK;
     static constexpr int KV_CHUNK = BLK * 128;    // BLK rows x 128 B
-    static constexpr int TMEM_S = 0;
-    static constexpr int TMEM_O = BLK;
-    static constexpr int TMEM_COLS = 256;
-    static_assert(BLK + D <= TMEM_COLS, "TMEM budget");
+    static constexpr int KV_STAGE = DC * KV_CHUNK;
+    static constexpr int P_STAGE = BC * Q_CHUNK;
+    static constexpr int NQ = (D == 128 && BLK == 128) ? 2 : 3;
+    static constexpr int NKV = (D == 128 && BLK == 128) ? 1 : 2;
+    static constexpr int NCTX = 4;
+    static constexpr int TMEM_S0 = 0, TMEM_O0 = 2 * BLK;   // S: 2 x BLK columns, O: 2 x D columns
+    static constexpr int TMEM_COLS = 512;
+    static_assert(2 * BLK + 2 * D <= TMEM_COLS, "TMEM budget");
+};
+
+constexpr int kSeqCache = 1024;   // sequences whose offsets the attention kernel keeps in smem
+
+struct TileCtx {
+    int64_t s0;        // first packed row of the block's sequence
+    int64_t j;         // block number within the sequence
+    int g, count, kvs, last_of_kv;
+    int32_t ent[128];
 };
 
 template <int D, int BLK, int G>
 struct AttnSmem {
     using A = AttnShape<D, BLK, G>;
-    alignas(1024) unsigned char q[A::DC * A::Q_CHUNK];
-    alignas(1024) unsigned char k[A::DC * A::KV_CHUNK];
-    alignas(1024) unsigned char v[A::DC * A::KV_CHUNK];
-    alignas(1024) unsigned char p[A::BC * A::Q_CHUNK];
-    alignas(8) uint64_t bar_kv, bar_q, bar_mma;
+    alignas(1024) unsigned char q[A::NQ][A::Q_STAGE];
+    alignas(1024) unsigned char kv[A::NKV][2][A::KV_STAGE];
+    alignas(1024) unsigned char p[2][A::P_STAGE];
+    TileCtx ctx[A::NCTX];
+    float2 ml[A::NCTX][128];
+    int32_t cu_blocks[kSeqCache + 1], cu_seqlens[kSeqCache + 1];   // small batches: sequence table
+    alignas(1024) unsigned char stage[4][32 * 128];   // epilogue: per-warp 32 rows x 64 columns (bf16)
+    alignas(8) uint64_t q_full[A::NQ], q_empty[A::NQ];
+    alignas(8) uint64_t kv_full[A::NKV], kv_empty[A::NKV];
+    alignas(8) uint64_t ctx_full[A::NCTX], ctx_empty[A::NCTX], ml_full[A::NCTX];
+    alignas(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2], o_empty[2];
+    alignas(8) uint64_t drain;
     uint32_t tmem_base;
     int fail;
-    int32_t ent[128];
 };
 
 struct PrefillBufs {
+    const __nv_bfloat16 *q;   // [T, Hq, D]
     const int32_t *entries;
     const int4 *tiles;
     const int32_t *n_tiles;   // device scalar (tile_off[L])
@@ -196,30 +226,61 @@ struct PrefillBufs {
     float *part_lse;          // [R, Hkv, k_tot, G]
 };
 
+// Bounded wait that records a failure in shared memory instead of hanging.
+__device__ __forceinline__ bool wait_or_fail(uint64_t *bar, uint32_t parity, int *fail) {
+    if (*(volatile int *)fail) return false;
+    if (!mbar_wait(bar, parity)) {
+        atomicExch(fail, 1);
+        return false;
+    }
+    return true;
+}
+
 template <int D, int BLK, int G>
-__global__ void __launch_bounds__(128) sparse_prefill_attn_kernel(Prob P, const __grid_constant__ CUtensorMap tm_q,
-                                                                  const __grid_constant__ CUtensorMap tm_k,
-                                                                  const __grid_constant__ CUtensorMap tm_v,
-                                                                  PrefillBufs W) {
+__global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, const __grid_constant__ CUtensorMap tm_q,
+                                                                     const __grid_constant__ CUtensorMap tm_k,
+                                                                     const __grid_constant__ CUtensorMap tm_v,
+                                                                     PrefillBufs W) {
     using A = AttnShape<D, BLK, G>;
     extern __shared__ unsigned char smem_raw[];
     AttnSmem<D, BLK, G> &S =
         *reinterpret_cast<AttnSmem<D, BLK, G> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        mbar_init(&S.bar_kv, 1);
-        mbar_init(&S.bar_q, 1);
-        mbar_init(&S.bar_mma, 1);
+        // q_full: one arrival per producer lane, each fired when that lane's copies have landed
+        for (int i = 0; i < A::NQ; ++i) { mbar_init(&S.q_full[i], 32); mbar_init(&S.q_empty[i], 1); }
+        for (int i = 0; i < A::NKV; ++i) { mbar_init(&S.kv_full[i], 1); mbar_init(&S.kv_empty[i], 1); }
+        for (int i = 0; i < A::NCTX; ++i) {
+            mbar_init(&S.ctx_full[i], 32);      // every producer lane publishes its own writes
+            mbar_init(&S.ctx_empty[i], 128);
+            mbar_init(&S.ml_full[i], 128);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.s_full[i], 1);
+            mbar_init(&S.s_empty[i], 128);
+            mbar_init(&S.p_full[i], 128);
+            mbar_init(&S.p_empty[i], 1);
+            mbar_init(&S.o_full[i], 1);
+            mbar_init(&S.o_empty[i], 128);
+        }
+        mbar_init(&S.drain, 1);
         S.fail = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
-    // rows of partially filled tiles read stale shared memory: start from zeros
-    for (int x = tid; x < (int)(sizeof(S.q) / 16); x += 128) reinterpret_cast<uint4 *>(S.q)[x] = make_uint4(0, 0, 0, 0);
-    if (warp == 0) {
+    // token slots a tile leaves empty read stale rows: start from zeros
+    for (int x = tid; x < (int)(sizeof(S.q) / 16); x += blockDim.x)
+        reinterpret_cast<uint4 *>(&S.q[0][0])[x] = make_uint4(0, 0, 0, 0);
+    const bool seq_cached = P.batch <= kSeqCache;
+    if (seq_cached)
+        for (int x = tid; x <= P.batch; x += blockDim.x) {
+            S.cu_blocks[x] = P.cu_blocks[x];
+            S.cu_seqlens[x] = P.cu_seqlens[x];
+        }
+    if (warp == 1) {
         tmem_alloc(&S.tmem_base, A::TMEM_COLS);
         tmem_relinquish();
     }
@@ -227,165 +288,318 @@ __global__ void __launch_bounds__(128) sparse_prefill_attn_kernel(Prob P, const 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
     const int n_tiles = *W.n_tiles;
-    const uint32_t idesc_s = idesc_bf16(128, BLK, 0, 0);
-    const uint32_t idesc_o = idesc_bf16(128, D, 0, 1);
-    uint32_t ph_kv = 0, ph_q = 0, ph_mma = 0;
-    bool kv_pending = false, q_pending = false;
-    int64_t cur_list = -1;
+    const int t_begin = (int)((int64_t)n_tiles * blockIdx.x / gridDim.x);
+    const int t_end = (int)((int64_t)n_tiles * (blockIdx.x + 1) / gridDim.x);
+    const int nt = t_end - t_begin;
 
-    const int u = tid / A::RPT, h = tid % A::RPT;   // this thread's row: token slot u, head h
-
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-        const int4 td = W.tiles[t];
-        const int64_t list = td.x;
-        const int first = td.y, count = td.z;
-        const int g = (int)(list / P.total_blocks);
-        const int64_t jglob = list % P.total_blocks;
-        const int b = seq_of_row(P.cu_blocks, P.batch, jglob);
-        const int64_t j = jglob - P.cu_blocks[b];
-        const int64_t s0 = P.cu_seqlens[b];
-        if (tid < count) S.ent[tid] = W.entries[first + tid];
-        __syncthreads();
-
-        if (tid == 0) {
-            if (list != cur_list) {
-                mbar_arrive_expect_tx(&S.bar_kv, 2 * A::DC * A::KV_CHUNK);
-#pragma unroll
-                for (int c = 0; c < A::DC; ++c) {
-                    tma_load_3d(S.k + c * A::KV_CHUNK, &tm_k, &S.bar_kv, c * 64, g, (int)(s0 + j * BLK));
-                    tma_load_3d(S.v + c * A::KV_CHUNK, &tm_v, &S.bar_kv, c * 64, g, (int)(s0 + j * BLK));
+    if (warp == 0) {
+        // ------------------------------------------------------------------ producer (whole warp:
+        // lane 0 waits and arrives, every lane loads entries and issues its token's Q gathers).
+        // Tile descriptors are held 32 at a time in the lanes (plus the next 32) and the next
+        // tile's entries are fetched one iteration ahead, so no global load sits on the chain.
+        const int32_t *cub = seq_cached ? S.cu_blocks : P.cu_blocks;
+        const int32_t *cus = seq_cached ? S.cu_seqlens : P.cu_seqlens;
+        int4 td_cur = make_int4(0, 0, 0, 0), td_nxt = make_int4(0, 0, 0, 0);
+        if (lane < nt) td_cur = W.tiles[t_begin + lane];
+        if (32 + lane < nt) td_nxt = W.tiles[t_begin + 32 + lane];
+        auto td_at = [&](int i, int base) -> int4 {   // descriptor of tile i, chunk base = 32*floor(i/32) of cur
+            const int r = i - base;
+            int4 v;
+            const bool in_cur = r < 32;
+            const int src = in_cur ? r : r - 32;
+            v.x = __shfl_sync(0xffffffffu, in_cur ? td_cur.x : td_nxt.x, src & 31);
+            v.y = __shfl_sync(0xffffffffu, in_cur ? td_cur.y : td_nxt.y, src & 31);
+            v.z = __shfl_sync(0xffffffffu, in_cur ? td_cur.z : td_nxt.z, src & 31);
+            v.w = 0;
+            return v;
+        };
+        int base = 0;
+        int4 td = nt > 0 ? td_at(0, 0) : make_int4(0, 0, 0, 0);
+        int ent = (nt > 0 && lane < td.z) ? W.entries[td.y + lane] : 0;
+        int64_t cur_list = -1;
+        int kv_uses = 0;
+        for (int i = 0; i < nt; ++i) {
+            // descriptor and entries of tile i+1 (issued now, consumed next iteration)
+            int4 td_n = make_int4(-1, 0, 0, 0);
+            if (i + 1 < nt) {
+                if (i + 1 - base >= 32 && (i + 1 - base) % 32 == 0) {
+                    // crossing into the next chunk of 32 descriptors
+                    base += 32;
+                    td_cur = td_nxt;
+                    td_nxt = (base + 32 + lane < nt) ? W.tiles[t_begin + base + 32 + lane] : make_int4(0, 0, 0, 0);
                 }
-                kv_pending = true;
+                td_n = td_at(i + 1, base);
             }
-            mbar_arrive_expect_tx(&S.bar_q, count * G * D * 2);
-            for (int x = 0; x < count; ++x) {
-                const int64_t p = P.row_begin + (S.ent[x] >> 8);
+            const int ent_n = (i + 1 < nt && lane < td_n.z) ? W.entries[td_n.y + lane] : 0;
+            const int64_t list = td.x;
+            const int cs = i % A::NCTX;
+            bool ok = lane == 0 ? wait_or_fail(&S.ctx_empty[cs], ((i / A::NCTX) & 1) ^ 1, &S.fail) : true;
+            if (!__all_sync(0xffffffffu, ok)) break;
+            TileCtx &c = S.ctx[cs];
+            const int64_t jglob = list % P.total_blocks;
+            const int b = seq_of_row(cub, P.batch, jglob);
+            const int g = (int)(list / P.total_blocks);
+            const int64_t j = jglob - cub[b];
+            const int64_t s0 = cus[b];
+            if (lane < td.z) c.ent[lane] = ent;
+            const bool new_kv = list != cur_list;
+            if (new_kv) {
+                ++kv_uses;
+                cur_list = list;
+            }
+            const int kvs = (kv_uses - 1) % A::NKV;
+            if (lane == 0) {
+                c.g = g;
+                c.j = j;
+                c.s0 = s0;
+                c.count = td.z;
+                c.kvs = kvs;
+                c.last_of_kv = (i + 1 == nt) || (td_n.x != list);   // next tile on another list
+            }
+            __syncwarp();
+            mbar_arrive(&S.ctx_full[cs]);
+            if (new_kv) {
+                ok = lane == 0 ? wait_or_fail(&S.kv_empty[kvs], (((kv_uses - 1) / A::NKV) & 1) ^ 1, &S.fail) : true;
+                if (!__all_sync(0xffffffffu, ok)) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&S.kv_full[kvs], 2 * A::KV_STAGE);
+                    const int row0 = (int)(s0 + j * BLK);
 #pragma unroll
-                for (int c = 0; c < A::DC; ++c)
-                    tma_load_3d(S.q + c * A::Q_CHUNK + x * A::RPT * 128, &tm_q, &S.bar_q, c * 64, g * G, (int)p);
+                    for (int cc = 0; cc < A::DC; ++cc) {
+                        tma_load_3d(S.kv[kvs][0] + cc * A::KV_CHUNK, &tm_k, &S.kv_full[kvs], cc * 64, g, row0);
+                        tma_load_3d(S.kv[kvs][1] + cc * A::KV_CHUNK, &tm_v, &S.kv_full[kvs], cc * 64, g, row0);
+                    }
+                }
             }
-            q_pending = true;
+            const int qs = i % A::NQ;
+            ok = lane == 0 ? wait_or_fail(&S.q_empty[qs], ((i / A::NQ) & 1) ^ 1, &S.fail) : true;
+            if (!__all_sync(0xffffffffu, ok)) break;
+            // gather the tile's query rows: 16-byte pieces, 512 contiguous bytes per warp instruction,
+            // written straight into the 128-byte-swizzled operand layout
+            {
+                const uint64_t keep = l2_policy_evict_last();   // the chunk's queries are gathered many times
+                unsigned char *qdst = S.q[qs];
+                constexpr int PIECES = G * D / 8;   // 16-byte pieces of one token's G heads
+                for (int u2 = 0; u2 < td.z; ++u2) {
+                    const int e2 = __shfl_sync(0xffffffffu, ent, u2);
+                    const __nv_bfloat16 *src = W.q + ((P.row_begin + (e2 >> 8)) * P.Hq + (int64_t)g * G) * D;
+#pragma unroll
+                    for (int pc = lane; pc < PIECES; pc += 32) {
+                        const int hh = pc / (D / 8), rem = pc % (D / 8);
+                        const int cc = rem / 8, qq = rem % 8;
+                        const int rrow = u2 * A::RPT + hh;
+                        cp_async_16_hint(qdst + cc * A::Q_CHUNK + sw128(rrow, qq), src + hh * D + rem * 8, keep);
+                    }
+                }
+                cp_async_arrive_noinc(&S.q_full[qs]);
+            }
+            td = td_n;
+            ent = ent_n;
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_bf16(128, BLK, 0, 0);
+            const uint32_t idesc_o = idesc_bf16(128, D, 0, 1);
+            int pend = -1, pend_kvs = 0, pend_last = 0;   // tile whose O = P V is not issued yet
+            int kv_uses = 0;
+            auto issue_pv = [&]() -> bool {
+                const int i = pend;
+                const int ps = i & 1;
+                if (!wait_or_fail(&S.p_full[ps], (i >> 1) & 1, &S.fail)) return false;
+                if (!wait_or_fail(&S.o_empty[ps], ((i >> 1) & 1) ^ 1, &S.fail)) return false;
+                tc_fence_after();
+                const uint32_t p0 = smem_u32(S.p[ps]), v0 = smem_u32(S.kv[pend_kvs][1]);
+#pragma unroll
+                for (int kc = 0; kc < A::BC; ++kc)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem + A::TMEM_O0 + ps * D, sdesc(p0 + kc * A::Q_CHUNK + kk * 32, 16, 1024),
+                                  sdesc(v0 + (kc * 64 + kk * 16) * 128, A::KV_CHUNK, 1024), idesc_o, (kc | kk) != 0);
+                umma_commit(&S.o_full[ps]);
+                umma_commit(&S.p_empty[ps]);
+                if (pend_last) umma_commit(&S.kv_empty[pend_kvs]);
+                pend = -1;
+                return true;
+            };
             bool ok = true;
-            if (kv_pending) { ok &= mbar_wait(&S.bar_kv, ph_kv); ph_kv ^= 1; kv_pending = false; }
-            ok &= mbar_wait(&S.bar_q, ph_q);
-            ph_q ^= 1;
-            q_pending = false;
-            if (!ok) S.fail = 1;
-            tc_fence_after();
-            const uint32_t q0 = smem_u32(S.q), k0 = smem_u32(S.k);
+            for (int i = 0; i < nt && ok; ++i) {
+                const int cs = i % A::NCTX;
+                if (!wait_or_fail(&S.ctx_full[cs], (i / A::NCTX) & 1, &S.fail)) { ok = false; break; }
+                const int kvs = S.ctx[cs].kvs;
+                const int last = S.ctx[cs].last_of_kv;
+                const bool new_kv = (i == 0) || pend_last;   // the producer reloads K/V exactly then
+                if (new_kv) {
+                    // with a single K/V stage the previous list's last P V must be issued before
+                    // the stage can be refilled
+                    if (A::NKV == 1 && pend >= 0 && !issue_pv()) { ok = false; break; }
+                    ++kv_uses;
+                    if (!wait_or_fail(&S.kv_full[kvs], ((kv_uses - 1) / A::NKV) & 1, &S.fail)) { ok = false; break; }
+                }
+                const int qs = i % A::NQ;
+                if (!wait_or_fail(&S.q_full[qs], (i / A::NQ) & 1, &S.fail)) { ok = false; break; }
+                fence_async_smem();   // the gathered rows were written by cp.async (generic proxy)
+                const int ts = i & 1;
+                if (!wait_or_fail(&S.s_empty[ts], ((i >> 1) & 1) ^ 1, &S.fail)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t q0 = smem_u32(S.q[qs]), k0 = smem_u32(S.kv[kvs][0]);
 #pragma unroll
-            for (int c = 0; c < A::DC; ++c)
+                for (int cc = 0; cc < A::DC; ++cc)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16(tmem + A::TMEM_S, sdesc(q0 + c * A::Q_CHUNK + kk * 32, 16, 1024),
-                              sdesc(k0 + c * A::KV_CHUNK + kk * 32, 16, 1024), idesc_s, (c | kk) != 0);
-            umma_commit(&S.bar_mma);
-        }
-        cur_list = list;
-
-        // this thread's row
-        const bool row_ok = (u < count) && (h < G);
-        int rr = 0, slot = 0;
-        int lim = BLK - 1;
-        if (row_ok) {
-            const int e = S.ent[u];
-            rr = e >> 8;
-            slot = e & 255;
-            const int64_t pos = P.row_begin + rr - s0;
-            if (pos / BLK == j) lim = (int)(pos - j * BLK);
-        }
-        if (!mbar_wait(&S.bar_mma, ph_mma)) S.fail = 1;
-        ph_mma ^= 1;
-        tc_fence_after();
-
-        // softmax over the block's keys (pass 1: max; pass 2: exponentials -> bf16 P tile)
-        float m2 = -INFINITY;
-#pragma unroll
-        for (int cc = 0; cc < BLK / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + A::TMEM_S + cc * 32, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int x = 0; x < 32; ++x)
-                if (cc * 32 + x <= lim) m2 = fmaxf(m2, __uint_as_float(v[x]) * P.scale_log2);
-        }
-        float l = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < BLK / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + A::TMEM_S + cc * 32, v);
-            tmem_ld_wait();
-            float pv[32];
-#pragma unroll
-            for (int x = 0; x < 32; ++x) {
-                pv[x] = (row_ok && cc * 32 + x <= lim) ? exp2f(__uint_as_float(v[x]) * P.scale_log2 - m2) : 0.f;
-                l += pv[x];
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem + A::TMEM_S0 + ts * BLK, sdesc(q0 + cc * A::Q_CHUNK + kk * 32, 16, 1024),
+                                  sdesc(k0 + cc * A::KV_CHUNK + kk * 32, 16, 1024), idesc_s, (cc | kk) != 0);
+                umma_commit(&S.s_full[ts]);
+                umma_commit(&S.q_empty[qs]);
+                if (pend >= 0 && !issue_pv()) { ok = false; break; }
+                pend = i;
+                pend_kvs = kvs;
+                pend_last = last;
             }
-            unsigned char *pc = S.p + (cc >> 1) * A::Q_CHUNK;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint4 w;
-                w.x = pack_bf16(pv[8 * q + 0], pv[8 * q + 1]);
-                w.y = pack_bf16(pv[8 * q + 2], pv[8 * q + 3]);
-                w.z = pack_bf16(pv[8 * q + 4], pv[8 * q + 5]);
-                w.w = pack_bf16(pv[8 * q + 6], pv[8 * q + 7]);
-                *reinterpret_cast<uint4 *>(pc + sw128(tid, (cc & 1) * 4 + q)) = w;
-            }
+            if (ok && pend >= 0) issue_pv();
+            umma_commit(&S.drain);   // arrives once every MMA issued above has completed
+            mbar_wait(&S.drain, 0);
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t p0 = smem_u32(S.p), v0 = smem_u32(S.v);
-#pragma unroll
-            for (int kc = 0; kc < A::BC; ++kc)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_bf16(tmem + A::TMEM_O, sdesc(p0 + kc * A::Q_CHUNK + kk * 32, 16, 1024),
-                              sdesc(v0 + (kc * 64 + kk * 16) * 128, A::KV_CHUNK, 1024), idesc_o, (kc | kk) != 0);
-            umma_commit(&S.bar_mma);
-        }
-        if (!mbar_wait(&S.bar_mma, ph_mma)) S.fail = 1;
-        ph_mma ^= 1;
-        tc_fence_after();
-
-        // epilogue: normalised partial O (bf16) and the block's log-sum-exp
-        const float inv_l = row_ok ? 1.f / l : 0.f;
-        const int64_t prow = (((int64_t)rr * P.Hkv + g) * P.k_tot + slot) * G + h;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + A::TMEM_O + cc * 32, v);
-            tmem_ld_wait();
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------------ softmax
+        const int row = tid - 128;
+        const int u = row / A::RPT, h = row % A::RPT;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        for (int i = 0; i < nt; ++i) {
+            const int cs = i % A::NCTX;
+            if (!__all_sync(0xffffffffu, wait_or_fail(&S.ctx_full[cs], (i / A::NCTX) & 1, &S.fail))) break;
+            const TileCtx &c = S.ctx[cs];
+            const bool row_ok = u < c.count && h < G;
+            int lim = BLK - 1;
             if (row_ok) {
-                uint4 *dst = reinterpret_cast<uint4 *>(W.part_o + prow * D + cc * 32);
+                const int64_t pos = P.row_begin + (c.ent[u] >> 8) - c.s0;
+                if (pos / BLK == c.j) lim = (int)(pos - c.j * BLK);
+            }
+            const int ts = i & 1;
+            if (!__all_sync(0xffffffffu, wait_or_fail(&S.s_full[ts], (i >> 1) & 1, &S.fail))) break;
+            tc_fence_after();
+            const uint32_t sbase = tmem + lane_base + A::TMEM_S0 + ts * BLK;
+            const bool masked = __any_sync(0xffffffffu, lim < BLK - 1);   // a local block in this warp
+            float smax = -INFINITY;
+#pragma unroll
+            for (int cc = 0; cc < BLK / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(sbase + cc * 32, v);
+                tmem_ld_wait();
+                if (masked) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        if (cc * 32 + x <= lim) smax = fmaxf(smax, __uint_as_float(v[x]));
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) smax = fmaxf(smax, __uint_as_float(v[x]));
+                }
+            }
+            const float m2 = smax * P.scale_log2;   // the scale is positive
+            if (!__all_sync(0xffffffffu, wait_or_fail(&S.p_empty[ts], ((i >> 1) & 1) ^ 1, &S.fail))) break;
+            // p = 2^(s * scale * log2 e - m); keys past the row's position get 2^-inf = 0.  Rows
+            // without a token are computed too: their O is never stored.
+            float l = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < BLK / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(sbase + cc * 32, v);
+                tmem_ld_wait();
+                float pv[32];
+                if (masked) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        pv[x] = ex2_approx(cc * 32 + x <= lim ? fmaf(__uint_as_float(v[x]), P.scale_log2, -m2) : -INFINITY);
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) pv[x] = ex2_approx(fmaf(__uint_as_float(v[x]), P.scale_log2, -m2));
+                }
+#pragma unroll
+                for (int x = 0; x < 32; ++x) l += pv[x];
+                unsigned char *pc = S.p[ts] + (cc >> 1) * A::Q_CHUNK;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     uint4 w;
-                    w.x = pack_bf16(__uint_as_float(v[8 * q + 0]) * inv_l, __uint_as_float(v[8 * q + 1]) * inv_l);
-                    w.y = pack_bf16(__uint_as_float(v[8 * q + 2]) * inv_l, __uint_as_float(v[8 * q + 3]) * inv_l);
-                    w.z = pack_bf16(__uint_as_float(v[8 * q + 4]) * inv_l, __uint_as_float(v[8 * q + 5]) * inv_l);
-                    w.w = pack_bf16(__uint_as_float(v[8 * q + 6]) * inv_l, __uint_as_float(v[8 * q + 7]) * inv_l);
-                    dst[q] = w;
+                    w.x = pack_bf16(pv[8 * q + 0], pv[8 * q + 1]);
+                    w.y = pack_bf16(pv[8 * q + 2], pv[8 * q + 3]);
+                    w.z = pack_bf16(pv[8 * q + 4], pv[8 * q + 5]);
+                    w.w = pack_bf16(pv[8 * q + 6], pv[8 * q + 7]);
+                    *reinterpret_cast<uint4 *>(pc + sw128(row, (cc & 1) * 4 + q)) = w;
                 }
             }
+            S.ml[cs][row] = make_float2(m2, l);
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&S.s_empty[ts]);
+            mbar_arrive(&S.p_full[ts]);
+            mbar_arrive(&S.ml_full[cs]);
         }
-        if (row_ok) W.part_lse[prow] = (m2 + __log2f(l)) * 0.69314718055994531f;
-        tc_fence_before();
-        __syncthreads();
-        if (S.fail) break;
-    }
-    if (S.fail && tid == 0) {
-        report(P.err, kErrTimeout);
-        if (kv_pending) mbar_wait(&S.bar_kv, ph_kv);
-        if (q_pending) mbar_wait(&S.bar_q, ph_q);
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------------ epilogue
+        const int row = tid - 256;
+        const int u = row / A::RPT, h = row % A::RPT;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        for (int i = 0; i < nt; ++i) {
+            const int cs = i % A::NCTX;
+            if (!__all_sync(0xffffffffu, wait_or_fail(&S.ctx_full[cs], (i / A::NCTX) & 1, &S.fail))) break;
+            if (!__all_sync(0xffffffffu, wait_or_fail(&S.ml_full[cs], (i / A::NCTX) & 1, &S.fail))) break;
+            const TileCtx &c = S.ctx[cs];
+            const bool row_ok = u < c.count && h < G;
+            const float2 ml = S.ml[cs][row];
+            int rr = 0, slot = 0;
+            if (row_ok) {
+                rr = c.ent[u] >> 8;
+                slot = c.ent[u] & 255;
+            }
+            const int os = i & 1;
+            if (!__all_sync(0xffffffffu, wait_or_fail(&S.o_full[os], (i >> 1) & 1, &S.fail))) break;
+            tc_fence_after();
+            const float inv_l = row_ok ? 1.f / ml.y : 0.f;
+            const int64_t prow = (((int64_t)rr * P.Hkv + c.g) * P.k_tot + slot) * G + h;
+            // each 64-column chunk: rows -> swizzled per-warp staging -> 4 full 128-byte lines per store
+            unsigned char *stg = S.stage[warp & 3];
+#pragma unroll
+            for (int cc = 0; cc < A::DC; ++cc) {
+                uint32_t v[2][32];
+                tmem_ld32(tmem + lane_base + A::TMEM_O0 + os * D + cc * 64, v[0]);
+                tmem_ld32(tmem + lane_base + A::TMEM_O0 + os * D + cc * 64 + 32, v[1]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const uint32_t *src = &v[q >> 2][(q & 3) * 8];
+                    uint4 w;
+                    w.x = pack_bf16(__uint_as_float(src[0]) * inv_l, __uint_as_float(src[1]) * inv_l);
+                    w.y = pack_bf16(__uint_as_float(src[2]) * inv_l, __uint_as_float(src[3]) * inv_l);
+                    w.z = pack_bf16(__uint_as_float(src[4]) * inv_l, __uint_as_float(src[5]) * inv_l);
+                    w.w = pack_bf16(__uint_as_float(src[6]) * inv_l, __uint_as_float(src[7]) * inv_l);
+                    *reinterpret_cast<uint4 *>(stg + sw128(lane, q)) = w;
+                }
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int r = 4 * k + (lane >> 3), q = lane & 7;
+                    const uint4 w = *reinterpret_cast<const uint4 *>(stg + sw128(r, q));
+                    const long long pr = __shfl_sync(0xffffffffu, (long long)prow, r);
+                    const bool okr = __shfl_sync(0xffffffffu, (int)row_ok, r) != 0;
+                    if (okr) st_global_cs(W.part_o + pr * D + cc * 64 + q * 8, w);   // streamed out, read once
+                }
+                __syncwarp();
+            }
+            if (row_ok) W.part_lse[prow] = (ml.x + __log2f(ml.y)) * 0.69314718055994531f;
+            tc_fence_before();
+            mbar_arrive(&S.o_empty[os]);
+            mbar_arrive(&S.ctx_empty[cs]);
+        }
     }
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, A::TMEM_COLS);
+    if (S.fail && tid == 0) report(P.err, kErrTimeout);
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, A::TMEM_COLS);
+    }
 }
 
 // ------------------------------------------------------------------------------- combine
@@ -419,7 +633,7 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(Prob P, const int3
             const int64_t pr = (w * P.k_tot + a) * G + h;
             const float wgt = __expf(part_lse[pr] - M);
             den += wgt;
-            uint4 raw = __ldg(reinterpret_cast<const uint4 *>(part_o + pr * D + d0));
+            uint4 raw = ld_global_cs(part_o + pr * D + d0);
             const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -478,11 +692,8 @@ static cudaError_t launch_attn_t(const Prob &P, const CUtensorMap &tq, const CUt
     auto kern = sparse_prefill_attn_kernel<D, BLK, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    int occ = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 128, smem);
-    if (e != cudaSuccess) return e;
-    occ = occ < 1 ? 1 : (occ > 2 ? 2 : occ);   // TMEM: 256 columns per CTA, 512 per SM
-    kern<<<num_sms * occ, 128, smem, st>>>(P, tq, tk, tv, W);
+    // one CTA per SM: it holds all 512 TMEM columns
+    kern<<<num_sms, 384, smem, st>>>(P, tq, tk, tv, W);
     return cudaGetLastError();
 }
 
@@ -507,7 +718,7 @@ static cudaError_t launch_combine_t(const Prob &P, const PrefillWs &w, void *O, 
     }
 
 cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                  const int32_t *block_idx, void *O, float *lse, void *ws, int num_sms,
+                                  const void *q, const int32_t *block_idx, void *O, float *lse, void *ws, int num_sms,
                                   cudaStream_t st) {
     const int64_t R = P.row_end - P.row_begin;
     if (R <= 0) return cudaSuccess;
@@ -534,7 +745,7 @@ cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CU
                                                                              w.tile_off, w.tiles);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    PrefillBufs W{w.entries, w.tiles, w.tile_off + L, w.part_o, w.part_lse};
+    PrefillBufs W{static_cast<const __nv_bfloat16 *>(q), w.entries, w.tiles, w.tile_off + L, w.part_o, w.part_lse};
     {
     ProfScope prof("prefill_attn", st);
     if (P.D == 128 && P.B == 64) { MSA_DISPATCH_G(P.G, e = launch_attn_t<128, 64, G_>(P, tq, tk, tv, W, num_sms, st)); }

@@ -37,8 +37,8 @@ struct PrefillWs {
 };
 PrefillWs prefill_ws_layout(const Prob &P, int64_t R, void *base);
 cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                  const int32_t *block_idx, void *O, float *lse, void *ws, int num_sms,
-                                  cudaStream_t st);
+                                  const void *q, const int32_t *block_idx, void *O, float *lse, void *ws,
+                                  int num_sms, cudaStream_t st);
 // attn_decode.cu
 size_t decode_ws_bytes(const Prob &P, int nct);
 void decode_geometry(const Prob &P, bool dense, int &nct, int &rounds);
