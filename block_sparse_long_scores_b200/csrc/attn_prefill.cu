@@ -163,11 +163,13 @@ __global__ void prefill_tiles_kernel(int64_t L, int tpt, const int32_t *__restri
 //
 // Warp-specialised persistent kernel; each CTA walks a contiguous range of tiles (tiles of one
 // list are adjacent, so a KV block is loaded once per CTA and list).  Roles:
-//   warp 0      producer: tile contexts, Q gathers (3-stage ring), K/V blocks (2 stages) by TMA
+//   warp 0      producer: tile contexts and K/V blocks (TMA, once per list)
+//   warps 2-3   query gather: cp.async of each token's G head rows into the swizzled operand
 //   warp 1      MMA issuer: S = Q K^T into one of 2 TMEM S buffers, O = P V into one of 2 TMEM O
 //               buffers; MMA1 of tile t+1 is issued before MMA2 of tile t
-//   warps 4-7   softmax: S (TMEM) -> row max/sum -> bf16 P tile (smem), one thread per row
-//   warps 8-11  epilogue: O (TMEM) -> normalised bf16 partial + lse -> global
+//   warps 4-7   softmax: S (TMEM) -> row max/sum -> bf16 P tile in shared memory, one thread per row
+//   warps 8-11  epilogue: O (TMEM) -> unnormalised bf16 partial + (max, sum) -> global through
+//               per-warp shared-memory staging
 // Hand-offs are mbarriers; "empty" barriers start free (first wait on parity 1 passes).
 
 template <int D, int BLK, int G>
@@ -181,15 +183,18 @@ struct AttnShape {
     static constexpr int KV_CHUNK = BLK * 128;    // BLK rows x 128 B
     static constexpr int KV_STAGE = DC * KV_CHUNK;
     static constexpr int P_STAGE = BC * Q_CHUNK;
-    static constexpr int NQ = (D == 128 && BLK == 128) ? 2 : 3;
-    static constexpr int NKV = (D == 128 && BLK == 128) ? 1 : 2;
-    static constexpr int NCTX = 4;
-    static constexpr int TMEM_S0 = 0, TMEM_O0 = 2 * BLK;   // S: 2 x BLK columns, O: 2 x D columns
+    // Query gathers arrive ~2 us after issue, so the ring keeps several in flight; K/V change only
+    // every few dozen tiles, so one K/V stage is enough where shared memory is short.
+    static constexpr int NQ = 4;
+    static constexpr int NKV = (D == 128) ? 1 : 2;
+    static constexpr int NCTX = 8;
+    // TMEM columns: S 2 x BLK, O 2 x D (fp32)
+    static constexpr int TMEM_S0 = 0, TMEM_O0 = 2 * BLK;
     static constexpr int TMEM_COLS = 512;
     static_assert(2 * BLK + 2 * D <= TMEM_COLS, "TMEM budget");
 };
 
-constexpr int kSeqCache = 1024;   // sequences whose offsets the attention kernel keeps in smem
+constexpr int kSeqCache = 256;   // sequences whose offsets the attention kernel keeps in smem
 
 struct TileCtx {
     int64_t s0;        // first packed row of the block's sequence
@@ -205,12 +210,12 @@ struct AttnSmem {
     alignas(1024) unsigned char kv[A::NKV][2][A::KV_STAGE];
     alignas(1024) unsigned char p[2][A::P_STAGE];
     TileCtx ctx[A::NCTX];
-    float2 ml[A::NCTX][128];
+    float2 ml[4][128];                     // softmax -> epilogue, ring of 4 (see ml_full)
     int32_t cu_blocks[kSeqCache + 1], cu_seqlens[kSeqCache + 1];   // small batches: sequence table
     alignas(1024) unsigned char stage[4][32 * 128];   // epilogue: per-warp 32 rows x 64 columns (bf16)
     alignas(8) uint64_t q_full[A::NQ], q_empty[A::NQ];
     alignas(8) uint64_t kv_full[A::NKV], kv_empty[A::NKV];
-    alignas(8) uint64_t ctx_full[A::NCTX], ctx_empty[A::NCTX], ml_full[A::NCTX];
+    alignas(8) uint64_t ctx_full[A::NCTX], ctx_empty[A::NCTX], ml_full[4];
     alignas(8) uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2], o_full[2], o_empty[2];
     alignas(8) uint64_t drain;
     uint32_t tmem_base;
@@ -222,8 +227,8 @@ struct PrefillBufs {
     const int32_t *entries;
     const int4 *tiles;
     const int32_t *n_tiles;   // device scalar (tile_off[L])
-    __nv_bfloat16 *part_o;    // [R, Hkv, k_tot, G, D]
-    float *part_lse;          // [R, Hkv, k_tot, G]
+    __nv_bfloat16 *part_o;    // [R, Hkv, k_tot, G, D], unnormalised: sum_t 2^(z_t - m) v_t
+    float2 *part_ml;          // [R, Hkv, k_tot, G]: (m, sum_t 2^(z_t - m)), z in log2 units
 };
 
 // Bounded wait that records a failure in shared memory instead of hanging.
@@ -248,14 +253,14 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        // q_full: one arrival per producer lane, each fired when that lane's copies have landed
-        for (int i = 0; i < A::NQ; ++i) { mbar_init(&S.q_full[i], 32); mbar_init(&S.q_empty[i], 1); }
+        // q_full: one arrival per gather lane (warps 2 and 3), fired when that lane's copies landed
+        for (int i = 0; i < A::NQ; ++i) { mbar_init(&S.q_full[i], 64); mbar_init(&S.q_empty[i], 1); }
         for (int i = 0; i < A::NKV; ++i) { mbar_init(&S.kv_full[i], 1); mbar_init(&S.kv_empty[i], 1); }
         for (int i = 0; i < A::NCTX; ++i) {
             mbar_init(&S.ctx_full[i], 32);      // every producer lane publishes its own writes
             mbar_init(&S.ctx_empty[i], 128);
-            mbar_init(&S.ml_full[i], 128);
         }
+        for (int i = 0; i < 4; ++i) mbar_init(&S.ml_full[i], 128);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.s_full[i], 1);
             mbar_init(&S.s_empty[i], 128);
@@ -338,9 +343,11 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
             bool ok = lane == 0 ? wait_or_fail(&S.ctx_empty[cs], ((i / A::NCTX) & 1) ^ 1, &S.fail) : true;
             if (!__all_sync(0xffffffffu, ok)) break;
             TileCtx &c = S.ctx[cs];
-            const int64_t jglob = list % P.total_blocks;
+            const uint32_t tb = (uint32_t)P.total_blocks;   // Hkv * total_blocks < 2^31 (host-checked)
+            const uint32_t g_u = (uint32_t)list / tb;
+            const int64_t jglob = (uint32_t)list - g_u * tb;
             const int b = seq_of_row(cub, P.batch, jglob);
-            const int g = (int)(list / P.total_blocks);
+            const int g = (int)g_u;
             const int64_t j = jglob - cub[b];
             const int64_t s0 = cus[b];
             if (lane < td.z) c.ent[lane] = ent;
@@ -373,30 +380,48 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
                     }
                 }
             }
-            const int qs = i % A::NQ;
-            ok = lane == 0 ? wait_or_fail(&S.q_empty[qs], ((i / A::NQ) & 1) ^ 1, &S.fail) : true;
-            if (!__all_sync(0xffffffffu, ok)) break;
-            // gather the tile's query rows: 16-byte pieces, 512 contiguous bytes per warp instruction,
-            // written straight into the 128-byte-swizzled operand layout
-            {
-                const uint64_t keep = l2_policy_evict_last();   // the chunk's queries are gathered many times
-                unsigned char *qdst = S.q[qs];
-                constexpr int PIECES = G * D / 8;   // 16-byte pieces of one token's G heads
-                for (int u2 = 0; u2 < td.z; ++u2) {
-                    const int e2 = __shfl_sync(0xffffffffu, ent, u2);
-                    const __nv_bfloat16 *src = W.q + ((P.row_begin + (e2 >> 8)) * P.Hq + (int64_t)g * G) * D;
-#pragma unroll
-                    for (int pc = lane; pc < PIECES; pc += 32) {
-                        const int hh = pc / (D / 8), rem = pc % (D / 8);
-                        const int cc = rem / 8, qq = rem % 8;
-                        const int rrow = u2 * A::RPT + hh;
-                        cp_async_16_hint(qdst + cc * A::Q_CHUNK + sw128(rrow, qq), src + hh * D + rem * 8, keep);
-                    }
-                }
-                cp_async_arrive_noinc(&S.q_full[qs]);
-            }
             td = td_n;
             ent = ent_n;
+        }
+    } else if (warp == 2 || warp == 3) {
+        // ------------------------------------------------------------------ query gather (warps 2, 3)
+        // Each warp copies half of the tile's tokens: the G head rows of a token are one contiguous
+        // run in Q; 16-byte pieces go straight to their 128-byte-swizzled operand positions.  A
+        // lane's pieces sit at the same offsets for every token, so they are computed once.
+        constexpr int PIECES = G * D / 8;                 // 16-byte pieces of one token's G heads
+        constexpr int PER_LANE = (PIECES + 31) / 32;
+        constexpr int HALF = (A::TPT + 1) / 2;
+        uint32_t dst_off[PER_LANE];
+        int src_off[PER_LANE];
+        bool has[PER_LANE];
+#pragma unroll
+        for (int k = 0; k < PER_LANE; ++k) {
+            const int pc = lane + 32 * k;
+            has[k] = pc < PIECES;
+            const int hh = pc / (D / 8), rem = pc % (D / 8);
+            dst_off[k] = (uint32_t)((rem / 8) * A::Q_CHUNK) + sw128(hh, rem % 8);   // token slot 0
+            src_off[k] = hh * D + rem * 8;
+        }
+        const uint64_t keep = l2_policy_evict_last();   // the chunk's queries are gathered many times
+        const int u0 = (warp - 2) * HALF;
+        for (int i = 0; i < nt; ++i) {
+            const int cs = i % A::NCTX;
+            bool ok = lane == 0 ? wait_or_fail(&S.ctx_full[cs], (i / A::NCTX) & 1, &S.fail) : true;
+            const int qs = i % A::NQ;
+            if (ok && lane == 0) ok = wait_or_fail(&S.q_empty[qs], ((i / A::NQ) & 1) ^ 1, &S.fail);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const TileCtx &c = S.ctx[cs];
+            const int count = c.count;
+            const int64_t qbase = P.row_begin * P.Hq + (int64_t)c.g * G;
+            unsigned char *qdst = S.q[qs];
+            for (int u = u0; u < u0 + HALF && u < count; ++u) {
+                const __nv_bfloat16 *src = W.q + (qbase + (int64_t)(c.ent[u] >> 8) * P.Hq) * D;
+                unsigned char *dst = qdst + u * (A::RPT * 128);
+#pragma unroll
+                for (int k = 0; k < PER_LANE; ++k)
+                    if (has[k]) cp_async_16_hint(dst + dst_off[k], src + src_off[k], keep);
+            }
+            cp_async_arrive_noinc(&S.q_full[qs]);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
@@ -482,39 +507,43 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
             tc_fence_after();
             const uint32_t sbase = tmem + lane_base + A::TMEM_S0 + ts * BLK;
             const bool masked = __any_sync(0xffffffffu, lim < BLK - 1);   // a local block in this warp
-            float smax = -INFINITY;
+            // S row -> registers with one wait (BLK/32 loads in flight together)
+            uint32_t sv[BLK / 32][32];
 #pragma unroll
-            for (int cc = 0; cc < BLK / 32; ++cc) {
-                uint32_t v[32];
-                tmem_ld32(sbase + cc * 32, v);
-                tmem_ld_wait();
-                if (masked) {
+            for (int cc = 0; cc < BLK / 32; ++cc) tmem_ld32(sbase + cc * 32, sv[cc]);
+            tmem_ld_wait();
+            float smax = -INFINITY;
+            if (masked) {
+#pragma unroll
+                for (int cc = 0; cc < BLK / 32; ++cc)
 #pragma unroll
                     for (int x = 0; x < 32; ++x)
-                        if (cc * 32 + x <= lim) smax = fmaxf(smax, __uint_as_float(v[x]));
-                } else {
+                        if (cc * 32 + x <= lim) smax = fmaxf(smax, __uint_as_float(sv[cc][x]));
+            } else {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) smax = fmaxf(smax, __uint_as_float(v[x]));
-                }
+                for (int cc = 0; cc < BLK / 32; ++cc)
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) smax = fmaxf(smax, __uint_as_float(sv[cc][x]));
             }
             const float m2 = smax * P.scale_log2;   // the scale is positive
+            // S is in registers: release the TMEM buffer for the next-but-one tile's S = Q K^T
+            tc_fence_before();
+            mbar_arrive(&S.s_empty[ts]);
             if (!__all_sync(0xffffffffu, wait_or_fail(&S.p_empty[ts], ((i >> 1) & 1) ^ 1, &S.fail))) break;
             // p = 2^(s * scale * log2 e - m); keys past the row's position get 2^-inf = 0.  Rows
             // without a token are computed too: their O is never stored.
             float l = 0.f;
 #pragma unroll
             for (int cc = 0; cc < BLK / 32; ++cc) {
-                uint32_t v[32];
-                tmem_ld32(sbase + cc * 32, v);
-                tmem_ld_wait();
                 float pv[32];
                 if (masked) {
 #pragma unroll
                     for (int x = 0; x < 32; ++x)
-                        pv[x] = ex2_approx(cc * 32 + x <= lim ? fmaf(__uint_as_float(v[x]), P.scale_log2, -m2) : -INFINITY);
+                        pv[x] = ex2_approx(cc * 32 + x <= lim ? fmaf(__uint_as_float(sv[cc][x]), P.scale_log2, -m2)
+                                                              : -INFINITY);
                 } else {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) pv[x] = ex2_approx(fmaf(__uint_as_float(v[x]), P.scale_log2, -m2));
+                    for (int x = 0; x < 32; ++x) pv[x] = ex2_approx(fmaf(__uint_as_float(sv[cc][x]), P.scale_log2, -m2));
                 }
 #pragma unroll
                 for (int x = 0; x < 32; ++x) l += pv[x];
@@ -529,67 +558,76 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
                     *reinterpret_cast<uint4 *>(pc + sw128(row, (cc & 1) * 4 + q)) = w;
                 }
             }
-            S.ml[cs][row] = make_float2(m2, l);
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(&S.s_empty[ts]);
+            S.ml[i & 3][row] = make_float2(m2, l);
+            fence_async_smem();   // P is read by the tensor core (async proxy)
             mbar_arrive(&S.p_full[ts]);
-            mbar_arrive(&S.ml_full[cs]);
+            mbar_arrive(&S.ml_full[i & 3]);
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------------ epilogue
         const int row = tid - 256;
         const int u = row / A::RPT, h = row % A::RPT;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        unsigned char *stg = S.stage[warp & 3];
+        const int Hkv = P.Hkv, k_tot = P.k_tot;
+        __nv_bfloat16 *const part_o = W.part_o;
+        float2 *const part_ml = W.part_ml;
         for (int i = 0; i < nt; ++i) {
             const int cs = i % A::NCTX;
-            if (!__all_sync(0xffffffffu, wait_or_fail(&S.ctx_full[cs], (i / A::NCTX) & 1, &S.fail))) break;
-            if (!__all_sync(0xffffffffu, wait_or_fail(&S.ml_full[cs], (i / A::NCTX) & 1, &S.fail))) break;
+            // ml_full is arrived by the softmax after it acquired this tile's context, so waiting on
+            // it also makes the context visible here
+            if (!__all_sync(0xffffffffu, wait_or_fail(&S.ml_full[i & 3], (i >> 2) & 1, &S.fail))) break;
             const TileCtx &c = S.ctx[cs];
             const bool row_ok = u < c.count && h < G;
-            const float2 ml = S.ml[cs][row];
+            const float2 ml = S.ml[i & 3][row];
             int rr = 0, slot = 0;
             if (row_ok) {
                 rr = c.ent[u] >> 8;
                 slot = c.ent[u] & 255;
             }
+            const int64_t prow = (((int64_t)rr * Hkv + c.g) * k_tot + slot) * G + h;
+            // destinations of the 8 rows this lane stores (rows 4k + lane/8), -1 if absent
+            __nv_bfloat16 *dst[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int r = 4 * k + (lane >> 3);
+                const long long pr = __shfl_sync(0xffffffffu, row_ok ? (long long)prow : -1ll, r);
+                dst[k] = pr >= 0 ? part_o + pr * D + (lane & 7) * 8 : nullptr;
+            }
             const int os = i & 1;
             if (!__all_sync(0xffffffffu, wait_or_fail(&S.o_full[os], (i >> 1) & 1, &S.fail))) break;
             tc_fence_after();
-            const float inv_l = row_ok ? 1.f / ml.y : 0.f;
-            const int64_t prow = (((int64_t)rr * P.Hkv + c.g) * P.k_tot + slot) * G + h;
             // each 64-column chunk: rows -> swizzled per-warp staging -> 4 full 128-byte lines per store
-            unsigned char *stg = S.stage[warp & 3];
 #pragma unroll
             for (int cc = 0; cc < A::DC; ++cc) {
                 uint32_t v[2][32];
                 tmem_ld32(tmem + lane_base + A::TMEM_O0 + os * D + cc * 64, v[0]);
                 tmem_ld32(tmem + lane_base + A::TMEM_O0 + os * D + cc * 64 + 32, v[1]);
                 tmem_ld_wait();
+                if (cc == A::DC - 1) {   // O is in registers: free the TMEM buffer early
+                    tc_fence_before();
+                    mbar_arrive(&S.o_empty[os]);
+                }
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const uint32_t *src = &v[q >> 2][(q & 3) * 8];
                     uint4 w;
-                    w.x = pack_bf16(__uint_as_float(src[0]) * inv_l, __uint_as_float(src[1]) * inv_l);
-                    w.y = pack_bf16(__uint_as_float(src[2]) * inv_l, __uint_as_float(src[3]) * inv_l);
-                    w.z = pack_bf16(__uint_as_float(src[4]) * inv_l, __uint_as_float(src[5]) * inv_l);
-                    w.w = pack_bf16(__uint_as_float(src[6]) * inv_l, __uint_as_float(src[7]) * inv_l);
+                    w.x = pack_bf16(__uint_as_float(src[0]), __uint_as_float(src[1]));
+                    w.y = pack_bf16(__uint_as_float(src[2]), __uint_as_float(src[3]));
+                    w.z = pack_bf16(__uint_as_float(src[4]), __uint_as_float(src[5]));
+                    w.w = pack_bf16(__uint_as_float(src[6]), __uint_as_float(src[7]));
                     *reinterpret_cast<uint4 *>(stg + sw128(lane, q)) = w;
                 }
                 __syncwarp();
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const int r = 4 * k + (lane >> 3), q = lane & 7;
-                    const uint4 w = *reinterpret_cast<const uint4 *>(stg + sw128(r, q));
-                    const long long pr = __shfl_sync(0xffffffffu, (long long)prow, r);
-                    const bool okr = __shfl_sync(0xffffffffu, (int)row_ok, r) != 0;
-                    if (okr) st_global_cs(W.part_o + pr * D + cc * 64 + q * 8, w);   // streamed out, read once
+                    const int r = 4 * k + (lane >> 3);
+                    const uint4 w = *reinterpret_cast<const uint4 *>(stg + sw128(r, lane & 7));
+                    if (dst[k]) st_global_cs(dst[k] + cc * 64, w);   // streamed out, read once
                 }
                 __syncwarp();
             }
-            if (row_ok) W.part_lse[prow] = (ml.x + __log2f(ml.y)) * 0.69314718055994531f;
-            tc_fence_before();
-            mbar_arrive(&S.o_empty[os]);
+            if (row_ok) part_ml[prow] = ml;   // (max in log2 units of the scaled logits, sum)
             mbar_arrive(&S.ctx_empty[cs]);
         }
     }
@@ -608,50 +646,93 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
 template <int D, int G>
 __global__ void __launch_bounds__(256) prefill_combine_kernel(Prob P, const int32_t *__restrict__ sanitized,
                                                               const __nv_bfloat16 *__restrict__ part_o,
-                                                              const float *__restrict__ part_lse,
+                                                              const float2 *__restrict__ part_ml,
                                                               __nv_bfloat16 *__restrict__ O, float *__restrict__ lse) {
+    // Partial a of a row holds O_a = sum_t 2^(z_t - m_a) v_t and l_a = sum_t 2^(z_t - m_a) (z in
+    // log2 units); the exact merge is O = sum_a 2^(m_a - M) O_a / sum_a 2^(m_a - M) l_a.
+    // NT threads per (row, kv head): thread t owns 8 dims of head t / (D/8); the D/8 threads of a
+    // head share the per-slot weights through shared memory.
     constexpr int NT = G * D / 8;
     constexpr int PAIRS = NT >= 256 ? 1 : 256 / NT;
+    constexpr int TPH = D / 8;                        // threads per head (8 or 16, within a warp)
+    extern __shared__ float wsh[];                    // [PAIRS][k_tot][G] weights, 0 for skipped slots
     const int tid = threadIdx.x;
     const int pair = tid / NT, t = tid % NT;
-    if (pair >= PAIRS) return;
+    const int k_tot = P.k_tot;
     const int64_t w = (int64_t)blockIdx.x * PAIRS + pair;
     const int64_t R = P.row_end - P.row_begin;
-    if (w >= R * P.Hkv) return;
-    const int64_t rr = w / P.Hkv;
-    const int g = (int)(w % P.Hkv);
-    const int h = t / (D / 8), d0 = (t % (D / 8)) * 8;
-    const int32_t *sel = sanitized + w * P.k_tot;
-    float M = -INFINITY;
-    for (int a = 0; a < P.k_tot; ++a)
-        if (sel[a] >= 0) M = fmaxf(M, part_lse[(w * P.k_tot + a) * G + h]);
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    float den = 0.f;
-    if (M > -INFINITY) {
-        for (int a = 0; a < P.k_tot; ++a) {
-            if (sel[a] < 0) continue;
-            const int64_t pr = (w * P.k_tot + a) * G + h;
-            const float wgt = __expf(part_lse[pr] - M);
-            den += wgt;
-            uint4 raw = ld_global_cs(part_o + pr * D + d0);
-            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+    const bool live = pair < PAIRS && w < R * P.Hkv;
+    const int h = t / TPH, d0 = (t % TPH) * 8, sub = t % TPH;
+    float *wp = wsh + pair * k_tot * G;
+    float M = -INFINITY, den = 0.f;
+    if (live) {
+        const int32_t *sel = sanitized + w * k_tot;
+        for (int a = sub; a < k_tot; a += TPH)
+            if (sel[a] >= 0) M = fmaxf(M, part_ml[(w * k_tot + a) * G + h].x);
+    }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float2 f = __bfloat1622float2(h2[q]);
-                acc[2 * q] = fmaf(wgt, f.x, acc[2 * q]);
-                acc[2 * q + 1] = fmaf(wgt, f.y, acc[2 * q + 1]);
+    for (int o = TPH / 2; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (live) {
+        const int32_t *sel = sanitized + w * k_tot;
+        for (int a = sub; a < k_tot; a += TPH) {
+            float wgt = 0.f;
+            if (sel[a] >= 0 && M > -INFINITY) {
+                const float2 ml = part_ml[(w * k_tot + a) * G + h];
+                wgt = ex2_approx(ml.x - M);
+                den = fmaf(wgt, ml.y, den);
+            }
+            wp[a * G + h] = wgt;
+        }
+    }
+#pragma unroll
+    for (int o = TPH / 2; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    __syncthreads();
+    if (!live) return;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const __nv_bfloat16 *src = part_o + (w * k_tot * G + h) * D + d0;
+    int a = 0;
+    for (; a + 4 <= k_tot; a += 4) {
+        uint4 raw[4];
+        float wg[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            wg[q] = wp[(a + q) * G + h];
+            raw[q] = wg[q] != 0.f ? ld_global_cs(src + (int64_t)(a + q) * G * D) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[q]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                acc[2 * e] = fmaf(wg[q], f.x, acc[2 * e]);
+                acc[2 * e + 1] = fmaf(wg[q], f.y, acc[2 * e + 1]);
             }
         }
     }
+    for (; a < k_tot; ++a) {
+        const float wg = wp[a * G + h];
+        if (wg == 0.f) continue;
+        const uint4 raw = ld_global_cs(src + (int64_t)a * G * D);
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h2[e]);
+            acc[2 * e] = fmaf(wg, f.x, acc[2 * e]);
+            acc[2 * e + 1] = fmaf(wg, f.y, acc[2 * e + 1]);
+        }
+    }
     const float inv = den > 0.f ? 1.f / den : 0.f;
-    const int64_t p = P.row_begin + rr;
+    const int64_t p = P.row_begin + w / P.Hkv;
+    const int g = (int)(w % P.Hkv);
     uint4 outv;
     outv.x = pack_bf16(acc[0] * inv, acc[1] * inv);
     outv.y = pack_bf16(acc[2] * inv, acc[3] * inv);
     outv.z = pack_bf16(acc[4] * inv, acc[5] * inv);
     outv.w = pack_bf16(acc[6] * inv, acc[7] * inv);
     *reinterpret_cast<uint4 *>(O + (p * P.Hq + (int64_t)g * G + h) * D + d0) = outv;
-    if (lse && d0 == 0) lse[p * P.Hq + (int64_t)g * G + h] = den > 0.f ? M + __logf(den) : -INFINITY;
+    if (lse && sub == 0)
+        lse[p * P.Hq + (int64_t)g * G + h] = den > 0.f ? (M + __log2f(den)) * 0.69314718055994531f : -INFINITY;
 }
 
 // ------------------------------------------------------------------------------ launchers
@@ -680,7 +761,7 @@ PrefillWs prefill_ws_layout(const Prob &P, int64_t R, void *base) {
     w.entries = (int32_t *)take(sizeof(int32_t) * E);
     w.tiles = (int4 *)take(sizeof(int4) * max_tiles);
     w.part_o = (__nv_bfloat16 *)take(sizeof(__nv_bfloat16) * E * P.G * P.D);
-    w.part_lse = (float *)take(sizeof(float) * E * P.G);
+    w.part_ml = (float2 *)take(sizeof(float2) * E * P.G);
     w.total = off;
     return w;
 }
@@ -702,8 +783,14 @@ static cudaError_t launch_combine_t(const Prob &P, const PrefillWs &w, void *O, 
     constexpr int NT = G * D / 8;
     constexpr int PAIRS = NT >= 256 ? 1 : 256 / NT;
     const int64_t n = (P.row_end - P.row_begin) * P.Hkv;
-    prefill_combine_kernel<D, G><<<(unsigned)ceil_div<int64_t>(n, PAIRS), 256, 0, st>>>(
-        P, w.sanitized, w.part_o, w.part_lse, (__nv_bfloat16 *)O, lse);
+    const size_t smem = sizeof(float) * PAIRS * P.k_tot * G;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_combine_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    prefill_combine_kernel<D, G><<<(unsigned)ceil_div<int64_t>(n, PAIRS), 256, smem, st>>>(
+        P, w.sanitized, w.part_o, w.part_ml, (__nv_bfloat16 *)O, lse);
     return cudaGetLastError();
 }
 
@@ -745,11 +832,10 @@ cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CU
                                                                              w.tile_off, w.tiles);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    PrefillBufs W{static_cast<const __nv_bfloat16 *>(q), w.entries, w.tiles, w.tile_off + L, w.part_o, w.part_lse};
+    PrefillBufs W{static_cast<const __nv_bfloat16 *>(q), w.entries, w.tiles, w.tile_off + L, w.part_o, w.part_ml};
     {
     ProfScope prof("prefill_attn", st);
     if (P.D == 128 && P.B == 64) { MSA_DISPATCH_G(P.G, e = launch_attn_t<128, 64, G_>(P, tq, tk, tv, W, num_sms, st)); }
-    else if (P.D == 128 && P.B == 128) { MSA_DISPATCH_G(P.G, e = launch_attn_t<128, 128, G_>(P, tq, tk, tv, W, num_sms, st)); }
     else if (P.D == 64 && P.B == 64) { MSA_DISPATCH_G(P.G, e = launch_attn_t<64, 64, G_>(P, tq, tk, tv, W, num_sms, st)); }
     else if (P.D == 64 && P.B == 128) { MSA_DISPATCH_G(P.G, e = launch_attn_t<64, 128, G_>(P, tq, tk, tv, W, num_sms, st)); }
     else return cudaErrorInvalidValue;

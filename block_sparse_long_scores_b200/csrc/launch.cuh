@@ -32,7 +32,7 @@ struct PrefillWs {
     int32_t *sanitized, *counts, *list_off, *cursor, *entries, *tile_off;
     int4 *tiles;
     __nv_bfloat16 *part_o;
-    float *part_lse;
+    float2 *part_ml;
     size_t total;
 };
 PrefillWs prefill_ws_layout(const Prob &P, int64_t R, void *base);

@@ -168,6 +168,9 @@ msa_status_t msa_select_topk(const msa_config_t *cfg, const msa_shape_t *shape,
  *  entries are skipped and flagged in *err_flag (nullable).
  *  Workspace: two-phase (file header); it grows with (row_end - row_begin), so long prefills are
  *  processed in row chunks.
+ *  Supported (head_dim, block_size): (64, 64), (64, 128), (128, 64); (128, 128) returns
+ *  MSA_ERR_UNSUPPORTED (the kernel's rings of query, key/value and probability tiles would not fit
+ *  an SM's shared memory).
  */
 msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t *shape,
                                      const void *q, const void *k, const void *v,
