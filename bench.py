@@ -137,32 +137,41 @@ class ClockSampler:
 
 
 class Dist:
-    def __init__(self, n_gpus: int):
+    """One process per GPU (torchrun); NCCL on GPUs, gloo for the CPU tests of this logic."""
+
+    def __init__(self, n_gpus: int, backend: str | None = None):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.on = self.world > 1
-        if self.on:
+        self.backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        self.device = torch.device("cuda", self.local) if self.backend == "nccl" else torch.device("cpu")
+        if self.backend == "nccl":
             torch.cuda.set_device(self.local)
-            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                                 device_id=torch.device("cuda", self.local))
-        elif torch.cuda.is_available():
-            torch.cuda.set_device(0)
+        if self.on:
+            kw = {"device_id": self.device} if self.backend == "nccl" else {}
+            torch.distributed.init_process_group(self.backend, timeout=datetime.timedelta(seconds=300), **kw)
 
     def barrier(self):
         if self.on:
             torch.distributed.barrier()
 
     def max(self, v: float) -> float:
+        """Largest value over ranks (device times are reported as the slowest rank's)."""
         if not self.on:
             return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.on:
             torch.distributed.destroy_process_group()
+
+
+def throughput(world: int, rows_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank's rows over the slowest rank's time (weak scaling)."""
+    return world * rows_per_rank * steps / (ms_max / 1000.0)
 
 
 def gpu_id(dist: Dist) -> str:
@@ -348,7 +357,7 @@ def main():
     msa.profile_reset()
     flops = selected_flops(pf)
     ms_step = ms / args.steps
-    value = dist.world * T * args.steps / (ms / 1000.0)
+    value = throughput(dist.world, T, args.steps, ms)
     attn_launch_ms = attn_ms / max(1, attn_n)
     flops_per_launch = flops / max(1, attn_n // args.steps)
     achieved = flops_per_launch / (attn_launch_ms / 1000.0) / 1e12
@@ -401,7 +410,7 @@ def end_to_end(args, dist, pf, x, T):
         lse_host.copy_(pf.lse, non_blocking=True)
 
     ms_e2e = timed(e2e_step, args.steps, 1, dist)
-    return {"value": dist.world * T * args.steps / (ms_e2e / 1000.0), "unit": "tokens/s",
+    return {"value": throughput(dist.world, T, args.steps, ms_e2e), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / args.steps}
 
 

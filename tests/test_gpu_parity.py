@@ -265,3 +265,109 @@ def test_decode_128k_full_size():
     w = WORKLOADS["decode_128k"]
     x = make_inputs(w, device=DEV)
     _decode_check(w, x)
+
+
+# ------------------------------------------------- full-size 1M and ragged, sampled rows
+# Host copies hold only what the oracle reads: Q rows of the sampled tokens (and, for decode, the
+# cache blocks the GPU selected); the rest of each host tensor is never touched.
+
+
+def _sparse_rows_cpu(t, rows):
+    out = torch.empty(t.shape, dtype=t.dtype)
+    idx = torch.as_tensor(rows, device=t.device)
+    out[torch.as_tensor(rows)] = t[idx].cpu()
+    return out
+
+
+def _prefill_sampled_check(w, x, rows, chunk_rows):
+    pf = Prefill(w, x, chunk_rows=chunk_rows)
+    S_gpu = np.zeros((len(rows), w.Hkv, pf.stride), np.float32)
+    qidx_gpu = torch.empty(pf.chunk, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV)
+    qidx_rows = np.zeros((len(rows), w.Hkv, w.d), np.uint16)
+    first = True
+    for r0, r1 in pf.chunks():
+        pf.index(r0, r1, compute_keys=first, q_idx_out=qidx_gpu)
+        first = False
+        pf.select(r0, r1)
+        pf.attend(r0, r1)
+        sel = (rows >= r0) & (rows < r1)
+        if sel.any():
+            loc = torch.as_tensor(rows[sel] - r0, device=DEV)
+            S_gpu[sel] = pf.scores[loc].cpu().numpy()
+            qidx_rows[sel] = _bits(qidx_gpu[loc])
+    torch.cuda.synchronize()
+    assert int(pf.err.item()) == 0
+    xc = {"q": _sparse_rows_cpu(x["q"], rows), "k": x["k"].cpu(), "v": x["v"].cpu(), "wq": x["wq"].cpu(),
+          "wk": x["wk"].cpu(), "cu_seqlens": x["cu_seqlens"].cpu(), "cu_blocks": x["cu_blocks"].cpu()}
+    sh = oracle_shape(w, xc)
+    kidx = _bits(pf.k_idx)
+    if "k_idx" in x:
+        assert np.array_equal(kidx, _bits(x["k_idx"]))
+    else:
+        _, khat = orc.block_keys(sh, xc["k"], xc["wk"])
+        check_bf16_near(kidx, khat, "k_idx")
+    check_bf16_near(qidx_rows, orc.index_query(sh, xc["q"], xc["wq"], rows)[1], "q_idx")
+    check_scores(w, xc, rows, S_gpu, orc.index_scores(sh, qidx_rows, kidx, rows, pf.stride))
+    sel_gpu = pf.block_idx[torch.as_tensor(rows, device=DEV)].cpu().numpy()
+    assert np.array_equal(sel_gpu, orc.select_topk_f32(sh, S_gpu, rows))
+    O_ref, L_ref = orc.sparse_attn(sh, xc["q"], xc["k"], xc["v"], sel_gpu, rows)
+    idx = torch.as_tensor(rows, device=DEV)
+    check_attention(pf.o[idx].float().cpu().numpy(), O_ref, pf.lse[idx].cpu().numpy(), L_ref)
+
+
+@pytest.mark.slow
+def test_prefill_1m_full_size_sampled():
+    w = WORKLOADS["prefill_1m"]
+    x = make_inputs(w, device=DEV)
+    _prefill_sampled_check(w, x, sample_rows(w, 192, seed=1), chunk_rows=16384)
+
+
+@pytest.mark.slow
+def test_ragged_prefill_full_size_sampled():
+    w = WORKLOADS["ragged_prefill"]
+    x = make_inputs(w, device=DEV)
+    _prefill_sampled_check(w, x, sample_rows(w, 1024, seed=2), chunk_rows=16384)
+
+
+def _decode_sampled_check(w, x):
+    dc = Decode(w, x)
+    qidx = torch.empty(w.batch, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV)
+    dc.run(q_idx_out=qidx)
+    torch.cuda.synchronize()
+    assert int(dc.err.item()) == 0
+    rows = np.arange(w.batch)
+    sel = dc.block_idx.cpu().numpy()
+    # host cache with only the selected blocks copied
+    kc = torch.empty(x["k"].shape, dtype=x["k"].dtype)
+    vc = torch.empty(x["v"].shape, dtype=x["v"].dtype)
+    for b in range(w.batch):
+        for g in range(w.Hkv):
+            for j in sel[b, g]:
+                if j >= 0:
+                    kc[b, g, j * w.B:(j + 1) * w.B] = x["k"][b, g, j * w.B:(j + 1) * w.B].cpu()
+                    vc[b, g, j * w.B:(j + 1) * w.B] = x["v"][b, g, j * w.B:(j + 1) * w.B].cpu()
+    xc = {"q": x["q"].cpu(), "k": kc, "v": vc, "wq": x["wq"].cpu(), "seqlens": x["seqlens"].cpu()}
+    sh = oracle_shape(w, xc)
+    kidx = _bits(dc.k_idx)
+    check_bf16_near(_bits(qidx), orc.index_query(sh, xc["q"], xc["wq"], rows)[1], "q_idx")
+    S_gpu = dc.scores.cpu().numpy()
+    check_scores(w, xc, rows, S_gpu, orc.index_scores(sh, _bits(qidx), kidx, rows, dc.stride))
+    assert np.array_equal(sel, orc.select_topk_f32(sh, S_gpu, rows))
+    O_ref, L_ref = orc.sparse_attn(sh, xc["q"], xc["k"], xc["v"], sel, rows)
+    check_attention(dc.o.float().cpu().numpy(), O_ref, dc.lse.cpu().numpy(), L_ref)
+
+
+@pytest.mark.slow
+def test_decode_1m_full_length():
+    # the 1M decode workload's length and selection (16384 blocks, 128 picks + sink + local) with 2
+    # of its 8 sequences, which keeps the host side small
+    w = WORKLOADS["decode_1m"].with_(seqlens=(1 << 20, (1 << 20) - 37))
+    x = make_inputs(w, device=DEV, seed=3)
+    _decode_sampled_check(w, x)
+
+
+@pytest.mark.slow
+def test_ragged_decode_full_size():
+    w = WORKLOADS["ragged_decode"]
+    x = make_inputs(w, device=DEV, seed=4)
+    _decode_sampled_check(w, x)
