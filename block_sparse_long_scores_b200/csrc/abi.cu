@@ -365,9 +365,7 @@ msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *
     if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
     if (shape->mode != MSA_DECODE || !workspace_bytes) return MSA_ERR_INVALID_ARG;
     const Prob P = make_prob(cfg, shape, 0, shape->batch, err_flag);
-    int nct, rounds;
-    decode_geometry(P, false, nct, rounds);
-    const size_t need = decode_ws_bytes(P, nct);
+    const size_t need = decode_stream_ws_bytes(P, num_sms());
     if (!workspace) {
         *workspace_bytes = need;
         return MSA_OK;
@@ -379,7 +377,8 @@ msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *
         return MSA_ERR_INVALID_ARG;
     CUtensorMap tq, tk, tv;
     if (!decode_maps(P, q, k_cache, v_cache, &tq, &tk, &tv)) return MSA_ERR_CUDA;
-    cudaError_t e = launch_decode(P, tq, tk, tv, block_idx, o, lse, workspace, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_decode_stream(P, tk, tv, q, block_idx, o, lse, workspace, num_sms(),
+                                         static_cast<cudaStream_t>(stream));
     return cuda_status(e, 1);
 }
 
@@ -434,9 +433,7 @@ msa_status_t msa_sparse_attn_decode_noalloc(const msa_config_t *cfg, const msa_s
     if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
     if (shape->mode != MSA_DECODE) return MSA_ERR_INVALID_ARG;
     const Prob P = make_prob(cfg, shape, 0, shape->batch, err_flag);
-    int nct, rounds;
-    decode_geometry(P, false, nct, rounds);
-    if (decode_ws_bytes(P, nct) > kNoAllocScratchBytes) return MSA_ERR_WORKSPACE;   // beyond the fixed scratch
+    if (decode_stream_ws_bytes(P, num_sms()) > kNoAllocScratchBytes) return MSA_ERR_WORKSPACE;   // beyond the fixed scratch
     if (!q || !k_cache || !v_cache || !block_idx || !o) return MSA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
         !aligned(block_idx, 4) || (lse && !aligned(lse, 4)))
@@ -445,8 +442,9 @@ msa_status_t msa_sparse_attn_decode_noalloc(const msa_config_t *cfg, const msa_s
     if (!scratch) return MSA_ERR_CUDA;
     CUtensorMap tq, tk, tv;
     if (!decode_maps(P, q, k_cache, v_cache, &tq, &tk, &tv)) return MSA_ERR_CUDA;
-    // launch_decode clears the split tickets in the scratch before its kernel runs
-    cudaError_t e = launch_decode(P, tq, tk, tv, block_idx, o, lse, scratch, static_cast<cudaStream_t>(stream));
+    // the launcher clears the merge tickets in the scratch before its kernel runs
+    cudaError_t e = launch_decode_stream(P, tk, tv, q, block_idx, o, lse, scratch, num_sms(),
+                                         static_cast<cudaStream_t>(stream));
     return cuda_status(e, 1);
 }
 

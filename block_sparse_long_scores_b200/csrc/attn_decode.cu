@@ -13,6 +13,8 @@
 // CTA of a (sequence, kv head) to finish (atomic ticket, no waiting) merges all splits:
 //   m = max_c m_c;  l = sum_c l_c 2^(m_c - m);  O = sum_c O_c 2^(m_c - m) / l;  lse = (m + log2 l) ln 2
 // (scores are kept in log2 units: t = scale * log2(e) * q.k).
+#include <algorithm>
+
 #include "launch.cuh"
 
 namespace msa {
@@ -344,6 +346,417 @@ cudaError_t launch_decode(const Prob &P, const CUtensorMap &tq, const CUtensorMa
     if (P.D == 128 && P.B == 128) return launch_dec_t<128, 128>(P, tq, tk, tv, block_idx, nct, rounds, W, O, lse, st);
     if (P.D == 64 && P.B == 64) return launch_dec_t<64, 64>(P, tq, tk, tv, block_idx, nct, rounds, W, O, lse, st);
     if (P.D == 64 && P.B == 128) return launch_dec_t<64, 128>(P, tq, tk, tv, block_idx, nct, rounds, W, O, lse, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace msa
+
+// ============================================================================================
+// Streaming sparse decode.
+//
+// The selected blocks of all (sequence, kv head) rows form one work list, item
+// x = (b * Hkv + g) * k_tot + slot.  A persistent grid splits the list into contiguous ranges; in a
+// CTA a producer warp streams the range's K/V blocks through an NS-stage TMA ring while three
+// consumer warps take items round robin, each keeping an online-softmax state per (b, g) segment
+// and flushing it as a split partial when its items move to the next segment.  The CTA that
+// completes a segment's ticket merges the segment's partials (same rule as above).
+// NS is a multiple of the consumer count, so a warp cycles through its own stages in order and
+// never waits on a stage's next fill before the previous one has landed (a parity wait cannot
+// tell the two apart).
+// ============================================================================================
+
+namespace msa {
+
+constexpr int kStreamConsumers = 3;
+
+template <int D, int BLK, int NS>
+struct StreamSmem {
+    static constexpr int DC = D / 64;
+    static constexpr int KV_CHUNK = BLK * 128;
+    alignas(1024) unsigned char k[NS][DC * KV_CHUNK];
+    alignas(1024) unsigned char v[NS][DC * KV_CHUNK];
+    alignas(8) uint64_t full[NS], empty[NS];
+    int js[NS];
+    int32_t row[256];     // sanitised block list of the producer's current (b, g)
+    int fail;
+    int last;
+};
+
+struct StreamBufs {
+    float *pm;            // [n_ctas, consumers, max_seg, 16]  running max (log2 units)
+    float *pl;            // [n_ctas, consumers, max_seg, 16]  running sum
+    float *po;            // [n_ctas, consumers, max_seg, 16, D] unnormalised output
+    int32_t *tickets;     // [batch * Hkv]
+    int max_seg;
+};
+
+__host__ __device__ __forceinline__ int64_t stream_begin(int64_t items, int64_t c, int64_t n) { return items * c / n; }
+// CTA whose range holds item x (largest c with stream_begin(c) <= x)
+__host__ __device__ __forceinline__ int64_t stream_cta_of(int64_t items, int64_t x, int64_t n) {
+    return ((x + 1) * n - 1) / items;
+}
+
+template <int D, int BLK, int NS>
+__global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_kernel(
+    Prob P, const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    const __nv_bfloat16 *__restrict__ Q, const int32_t *__restrict__ block_idx, StreamBufs W,
+    __nv_bfloat16 *__restrict__ O, float *__restrict__ lse) {
+    using SM = StreamSmem<D, BLK, NS>;
+    constexpr int DC = SM::DC;
+    extern __shared__ unsigned char smem_raw[];
+    SM &S = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t items = (int64_t)P.batch * P.Hkv * P.k_tot;
+    const int64_t c = blockIdx.x, nc = gridDim.x;
+    const int64_t x0 = stream_begin(items, c, nc), x1 = stream_begin(items, c + 1, nc);
+    const int n = (int)(x1 - x0);
+    const int k_tot = P.k_tot;
+    const int64_t bg_first = x0 / k_tot;
+    const int nseg = n > 0 ? (int)((x1 - 1) / k_tot - bg_first + 1) : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&S.full[s], 1);
+            mbar_init(&S.empty[s], 1);
+        }
+        S.fail = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == kStreamConsumers) {
+        // ------------------------------------------------------------------ producer (warp)
+        // Entering a (b, g) row, the warp loads its block list once and sanitises it (out of range,
+        // future or repeated -> -1, flagged); lane 0 then streams the row's blocks of this range.
+        int64_t cur_bg = -1;
+        for (int k = 0; k < n; ++k) {
+            const int64_t x = x0 + k;
+            const int64_t bg = x / k_tot;
+            const int a = (int)(x - bg * k_tot);
+            if (bg != cur_bg) {
+                __syncwarp();
+                const int b = (int)(bg / P.Hkv);
+                const int64_t i = ((int64_t)P.seqlens[b] - 1) / BLK;
+                const int32_t *row = block_idx + bg * k_tot;
+                bool canon = true;
+                int bad = 0;
+                for (int q = lane; q < k_tot; q += 32) {
+                    int j = row[q];
+                    if (j < -1 || j > i) { bad |= kErrBlockRange; j = -1; }
+                    S.row[q] = j;
+                }
+                __syncwarp();
+                for (int q = lane; q < k_tot; q += 32)   // valid entries strictly ascending, then -1 only
+                    if (q > 0 && S.row[q] >= 0 && !(S.row[q - 1] >= 0 && S.row[q - 1] < S.row[q])) canon = false;
+                canon = __all_sync(0xffffffffu, canon);
+                if (!canon) {
+                    int32_t keep[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        const int q = lane + 32 * t;
+                        keep[t] = q < k_tot ? S.row[q] : -1;
+                        if (keep[t] >= 0)
+                            for (int r = 0; r < q; ++r)
+                                if (S.row[r] == keep[t]) { bad |= kErrDuplicate; keep[t] = -1; break; }
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int t = 0; t < 8; ++t)
+                        if (lane + 32 * t < k_tot) S.row[lane + 32 * t] = keep[t];
+                }
+                if (bad) report(P.err, bad);
+                __syncwarp();
+                cur_bg = bg;
+            }
+            if (lane == 0) {
+                const int s = k % NS;
+                if (!mbar_wait(&S.empty[s], ((k / NS) & 1) ^ 1)) S.fail = 1;
+                const int j = S.row[a];
+                S.js[s] = j;
+                if (j >= 0) {
+                    mbar_arrive_expect_tx(&S.full[s], 2 * DC * SM::KV_CHUNK);
+                    const int row0 = (int)(bg * P.Lmax + (int64_t)j * BLK);
+#pragma unroll
+                    for (int cc = 0; cc < DC; ++cc) {
+                        tma_load_2d(S.k[s] + cc * SM::KV_CHUNK, &tm_k, &S.full[s], cc * 64, row0);
+                        tma_load_2d(S.v[s] + cc * SM::KV_CHUNK, &tm_v, &S.full[s], cc * 64, row0);
+                    }
+                } else {
+                    mbar_arrive(&S.full[s]);   // nothing to load: the slot is skipped
+                }
+            }
+            if (__any_sync(0xffffffffu, S.fail != 0)) break;
+        }
+    } else {
+        // ------------------------------------------------------------------ consumers
+        float m_r[2], l_r[2];
+        float o[D / 8][4];
+        uint32_t qf[D / 16][4];
+        int cur = -1;   // current segment (b, g) - bg_first
+        auto reset = [&]() {
+            m_r[0] = m_r[1] = -INFINITY;
+            l_r[0] = l_r[1] = 0.f;
+#pragma unroll
+            for (int dt = 0; dt < D / 8; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+        };
+        auto flush = [&](int seg) {
+            const int64_t slot = ((c * kStreamConsumers + warp) * W.max_seg + seg) * 16;
+            float l0 = l_r[0], l1 = l_r[1];
+            l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+            l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+            const int r0 = lane >> 2;
+            if ((lane & 3) == 0) {
+                W.pm[slot + r0] = m_r[0];
+                W.pm[slot + r0 + 8] = m_r[1];
+                W.pl[slot + r0] = l0;
+                W.pl[slot + r0 + 8] = l1;
+            }
+#pragma unroll
+            for (int dt = 0; dt < D / 8; ++dt) {
+                const int col = dt * 8 + 2 * (lane & 3);
+                *reinterpret_cast<float2 *>(W.po + (slot + r0) * D + col) = make_float2(o[dt][0], o[dt][1]);
+                *reinterpret_cast<float2 *>(W.po + (slot + r0 + 8) * D + col) = make_float2(o[dt][2], o[dt][3]);
+            }
+        };
+        auto load_q = [&](int64_t bg) {
+            const int b = (int)(bg / P.Hkv), g = (int)(bg % P.Hkv);
+            const int r0 = lane >> 2, r1 = r0 + 8;
+            const __nv_bfloat16 *q0 = Q + ((int64_t)b * P.Hq + (int64_t)g * P.G + r0) * D;
+            const __nv_bfloat16 *q1 = Q + ((int64_t)b * P.Hq + (int64_t)g * P.G + r1) * D;
+            const bool ok0 = r0 < P.G, ok1 = r1 < P.G;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const int col = ks * 16 + 2 * (lane & 3);
+                qf[ks][0] = ok0 ? *reinterpret_cast<const uint32_t *>(q0 + col) : 0u;
+                qf[ks][1] = ok1 ? *reinterpret_cast<const uint32_t *>(q1 + col) : 0u;
+                qf[ks][2] = ok0 ? *reinterpret_cast<const uint32_t *>(q0 + col + 8) : 0u;
+                qf[ks][3] = ok1 ? *reinterpret_cast<const uint32_t *>(q1 + col + 8) : 0u;
+            }
+        };
+        reset();
+        for (int k = warp; k < n; k += kStreamConsumers) {
+            const int s = k % NS;
+            if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (k / NS) & 1))) {
+                if (lane == 0) S.fail = 1;
+                break;
+            }
+            const int64_t x = x0 + k;
+            const int64_t bg = x / k_tot;
+            const int seg = (int)(bg - bg_first);
+            if (seg != cur) {
+                if (cur >= 0) flush(cur);
+                for (int z = cur + 1; z < seg; ++z) {   // segments this warp never touched
+                    reset();
+                    flush(z);
+                }
+                reset();
+                load_q(bg);
+                cur = seg;
+            }
+            const int j = S.js[s];
+            if (j >= 0) {
+                const int b = (int)(bg / P.Hkv);
+                const int64_t pos = (int64_t)P.seqlens[b] - 1;
+                const int64_t i = pos / BLK;
+                const uint32_t k_base = smem_u32(S.k[s]), v_base = smem_u32(S.v[s]);
+                float sc[BLK / 8][4];
+#pragma unroll
+                for (int nt = 0; nt < BLK / 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const int cch = ks / 4;
+#pragma unroll
+                    for (int nt = 0; nt < BLK / 8; nt += 2) {
+                        const int mi = lane >> 3;
+                        const int key = (nt + (mi >> 1)) * 8 + (lane & 7);
+                        const int ch = (ks * 2 + (mi & 1)) & 7;
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(k_base + cch * SM::KV_CHUNK + sw128(key, ch), b0, b1, b2, b3);
+                        mma_bf16_16816(sc[nt], qf[ks], b0, b1);
+                        mma_bf16_16816(sc[nt + 1], qf[ks], b2, b3);
+                    }
+                }
+                const int lim = (j == i) ? (int)(pos - (int64_t)j * BLK) : BLK - 1;
+                float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+                for (int nt = 0; nt < BLK / 8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int key = nt * 8 + 2 * (lane & 3) + (e & 1);
+                        const float t = key <= lim ? sc[nt][e] * P.scale_log2 : -INFINITY;
+                        sc[nt][e] = t;
+                        mx[e >> 1] = fmaxf(mx[e >> 1], t);
+                    }
+                float alpha[2];
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
+                    mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
+                    const float m_new = fmaxf(m_r[rr], mx[rr]);
+                    alpha[rr] = ex2_approx(m_r[rr] - m_new);
+                    m_r[rr] = m_new;
+                }
+                float ls[2] = {0.f, 0.f};
+#pragma unroll
+                for (int nt = 0; nt < BLK / 8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float p = ex2_approx(sc[nt][e] - m_r[e >> 1]);
+                        sc[nt][e] = p;
+                        ls[e >> 1] += p;
+                    }
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) l_r[rr] = l_r[rr] * alpha[rr] + ls[rr];
+#pragma unroll
+                for (int dt = 0; dt < D / 8; ++dt) {
+                    o[dt][0] *= alpha[0];
+                    o[dt][1] *= alpha[0];
+                    o[dt][2] *= alpha[1];
+                    o[dt][3] *= alpha[1];
+                }
+#pragma unroll
+                for (int kt = 0; kt < BLK / 16; ++kt) {
+                    uint32_t pa[4];
+                    pa[0] = pack_bf16(sc[2 * kt][0], sc[2 * kt][1]);
+                    pa[1] = pack_bf16(sc[2 * kt][2], sc[2 * kt][3]);
+                    pa[2] = pack_bf16(sc[2 * kt + 1][0], sc[2 * kt + 1][1]);
+                    pa[3] = pack_bf16(sc[2 * kt + 1][2], sc[2 * kt + 1][3]);
+#pragma unroll
+                    for (int dt = 0; dt < D / 8; dt += 2) {
+                        const int mi = lane >> 3;
+                        const int key = kt * 16 + (mi & 1) * 8 + (lane & 7);
+                        const int dch = dt + (mi >> 1);
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_t(v_base + (dch >> 3) * SM::KV_CHUNK + sw128(key, dch & 7), b0, b1, b2, b3);
+                        mma_bf16_16816(o[dt], pa, b0, b1);
+                        mma_bf16_16816(o[dt + 1], pa, b2, b3);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.empty[s]);
+        }
+        if (cur >= 0) flush(cur);
+        for (int z = cur + 1; z < nseg; ++z) {
+            reset();
+            flush(z);
+        }
+    }
+
+    // every partial of this CTA is written: take the tickets of its segments; the CTA that
+    // completes a segment merges it
+    __threadfence();
+    __syncthreads();
+    for (int seg = 0; seg < nseg; ++seg) {
+        const int64_t bg = bg_first + seg;
+        const int64_t c_first = stream_cta_of(items, bg * k_tot, nc);
+        const int64_t c_last = stream_cta_of(items, (bg + 1) * k_tot - 1, nc);
+        if (tid == 0) S.last = atomicAdd(&W.tickets[bg], 1) == (int)(c_last - c_first);
+        __syncthreads();
+        if (S.last) {
+            __threadfence();
+            const int b = (int)(bg / P.Hkv), g = (int)(bg % P.Hkv);
+            for (int e = tid; e < P.G * D; e += blockDim.x) {
+                const int r = e / D, col = e % D;
+                float M = -INFINITY;
+                for (int64_t cc = c_first; cc <= c_last; ++cc) {
+                    const int sg = (int)(bg - stream_begin(items, cc, nc) / k_tot);
+                    for (int w = 0; w < kStreamConsumers; ++w)
+                        M = fmaxf(M, __ldcg(&W.pm[((cc * kStreamConsumers + w) * W.max_seg + sg) * 16 + r]));
+                }
+                float L = 0.f, acc = 0.f;
+                if (M > -INFINITY) {
+                    for (int64_t cc = c_first; cc <= c_last; ++cc) {
+                        const int sg = (int)(bg - stream_begin(items, cc, nc) / k_tot);
+                        for (int w = 0; w < kStreamConsumers; ++w) {
+                            const int64_t sl = ((cc * kStreamConsumers + w) * W.max_seg + sg) * 16 + r;
+                            const float mm = __ldcg(&W.pm[sl]);
+                            if (mm == -INFINITY) continue;
+                            const float f = ex2_approx(mm - M);
+                            L += __ldcg(&W.pl[sl]) * f;
+                            acc += __ldcg(&W.po[sl * D + col]) * f;
+                        }
+                    }
+                }
+                const int64_t orow = (int64_t)b * P.Hq + (int64_t)g * P.G + r;
+                O[orow * D + col] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+                if (lse && col == 0) lse[orow] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+            }
+            if (tid == 0) W.tickets[bg] = 0;
+        }
+        __syncthreads();
+    }
+    if (S.fail && tid == 0) report(P.err, kErrTimeout);
+}
+
+template <int D, int BLK>
+struct StreamCfg {
+    // a multiple of the consumer count: two stages per consumer warp where 32 KB blocks allow it
+    static constexpr int NS = (2 * D * BLK * 2 <= 32768) ? 2 * kStreamConsumers : kStreamConsumers;
+    static size_t smem() { return sizeof(StreamSmem<D, BLK, NS>) + 1024; }
+};
+
+// Grid, segment bound and workspace of the streaming decode.
+void decode_stream_geometry(const Prob &P, int num_sms, int &n_ctas, int &max_seg) {
+    size_t smem = 0;
+    if (P.D == 128 && P.B == 64) smem = StreamCfg<128, 64>::smem();
+    else if (P.D == 128 && P.B == 128) smem = StreamCfg<128, 128>::smem();
+    else if (P.D == 64 && P.B == 64) smem = StreamCfg<64, 64>::smem();
+    else smem = StreamCfg<64, 128>::smem();
+    const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(2, (size_t)(227 * 1024) / smem));
+    static_assert(StreamCfg<128, 64>::NS % kStreamConsumers == 0 && StreamCfg<128, 128>::NS % kStreamConsumers == 0,
+                  "stage count must be a multiple of the consumer warps");
+    const int64_t items = (int64_t)P.batch * P.Hkv * P.k_tot;
+    n_ctas = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms * per_sm, items));
+    const int64_t per_cta = ceil_div<int64_t>(items, n_ctas);
+    max_seg = (int)(ceil_div<int64_t>(per_cta, P.k_tot) + 1);
+}
+
+size_t decode_stream_ws_bytes(const Prob &P, int num_sms) {
+    int n_ctas, max_seg;
+    decode_stream_geometry(P, num_sms, n_ctas, max_seg);
+    auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t rows = (size_t)n_ctas * kStreamConsumers * max_seg * 16;
+    return 2 * a(sizeof(float) * rows) + a(sizeof(float) * rows * P.D) + a(sizeof(int32_t) * P.batch * P.Hkv);
+}
+
+template <int D, int BLK>
+static cudaError_t launch_stream_t(const Prob &P, const CUtensorMap &tk, const CUtensorMap &tv, const void *q,
+                                   const int32_t *block_idx, const StreamBufs &W, int n_ctas, void *O, float *lse,
+                                   cudaStream_t st) {
+    constexpr int NS = StreamCfg<D, BLK>::NS;
+    const size_t smem = StreamCfg<D, BLK>::smem();
+    auto kern = decode_stream_kernel<D, BLK, NS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<n_ctas, 32 * (kStreamConsumers + 1), smem, st>>>(P, tk, tv, (const __nv_bfloat16 *)q, block_idx, W,
+                                                           (__nv_bfloat16 *)O, lse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_stream(const Prob &P, const CUtensorMap &tk, const CUtensorMap &tv, const void *q,
+                                 const int32_t *block_idx, void *O, float *lse, void *ws, int num_sms,
+                                 cudaStream_t st) {
+    int n_ctas, max_seg;
+    decode_stream_geometry(P, num_sms, n_ctas, max_seg);
+    auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t rows = (size_t)n_ctas * kStreamConsumers * max_seg * 16;
+    char *base = static_cast<char *>(ws);
+    StreamBufs W;
+    W.pm = reinterpret_cast<float *>(base);
+    W.pl = reinterpret_cast<float *>(base + a(sizeof(float) * rows));
+    W.po = reinterpret_cast<float *>(base + 2 * a(sizeof(float) * rows));
+    W.tickets = reinterpret_cast<int32_t *>(base + 2 * a(sizeof(float) * rows) + a(sizeof(float) * rows * P.D));
+    W.max_seg = max_seg;
+    cudaError_t e = cudaMemsetAsync(W.tickets, 0, sizeof(int32_t) * P.batch * P.Hkv, st);
+    if (e != cudaSuccess) return e;
+    ProfScope prof("decode_attn", st);
+    if (P.D == 128 && P.B == 64) return launch_stream_t<128, 64>(P, tk, tv, q, block_idx, W, n_ctas, O, lse, st);
+    if (P.D == 128 && P.B == 128) return launch_stream_t<128, 128>(P, tk, tv, q, block_idx, W, n_ctas, O, lse, st);
+    if (P.D == 64 && P.B == 64) return launch_stream_t<64, 64>(P, tk, tv, q, block_idx, W, n_ctas, O, lse, st);
+    if (P.D == 64 && P.B == 128) return launch_stream_t<64, 128>(P, tk, tv, q, block_idx, W, n_ctas, O, lse, st);
     return cudaErrorInvalidValue;
 }
 
