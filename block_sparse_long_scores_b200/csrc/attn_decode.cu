@@ -355,19 +355,19 @@ cudaError_t launch_decode(const Prob &P, const CUtensorMap &tq, const CUtensorMa
 // Streaming sparse decode.
 //
 // The selected blocks of all (sequence, kv head) rows form one work list, item
-// x = (b * Hkv + g) * k_tot + slot.  A persistent grid splits the list into contiguous ranges; in a
-// CTA a producer warp streams the range's K/V blocks through an NS-stage TMA ring while three
-// consumer warps take items round robin, each keeping an online-softmax state per (b, g) segment
-// and flushing it as a split partial when its items move to the next segment.  The CTA that
-// completes a segment's ticket merges the segment's partials (same rule as above).
-// NS is a multiple of the consumer count, so a warp cycles through its own stages in order and
-// never waits on a stage's next fill before the previous one has landed (a parity wait cannot
-// tell the two apart).
+// x = (b * Hkv + g) * k_tot + slot.  A persistent grid splits the list into contiguous ranges.  In a
+// CTA a producer warp streams the range's K/V blocks through an NS-stage TMA ring and the four
+// consumer warps all read every stage: warp w takes keys [w BLK/4, (w+1) BLK/4) of the block, so the
+// chain of dependent tensor-core and softmax steps per block is a quarter of a whole block's.  Each
+// warp keeps an online-softmax state for the current (b, g) segment; when the range moves to the
+// next segment the four states are merged in shared memory into one split partial (m, l, O) of the
+// segment.  The CTA that completes a segment's ticket merges the segment's partials (same rule as
+// above).
 // ============================================================================================
 
 namespace msa {
 
-constexpr int kStreamConsumers = 3;
+constexpr int kStreamConsumers = 4;
 
 template <int D, int BLK, int NS>
 struct StreamSmem {
@@ -375,6 +375,9 @@ struct StreamSmem {
     static constexpr int KV_CHUNK = BLK * 128;
     alignas(1024) unsigned char k[NS][DC * KV_CHUNK];
     alignas(1024) unsigned char v[NS][DC * KV_CHUNK];
+    float ob[16][D + 8];       // consumer warps' O merged at a flush (rows padded: no bank conflicts)
+    float mw[kStreamConsumers][16], lw[kStreamConsumers][16];
+    int lastf[32];             // tickets taken: this CTA merges the segment
     alignas(8) uint64_t full[NS], empty[NS];
     int js[NS];
     int32_t row[256];     // sanitised block list of the producer's current (b, g)
@@ -383,9 +386,9 @@ struct StreamSmem {
 };
 
 struct StreamBufs {
-    float *pm;            // [n_ctas, consumers, max_seg, 16]  running max (log2 units)
-    float *pl;            // [n_ctas, consumers, max_seg, 16]  running sum
-    float *po;            // [n_ctas, consumers, max_seg, 16, D] unnormalised output
+    float *pm;            // [n_ctas, max_seg, 16]  running max (log2 units)
+    float *pl;            // [n_ctas, max_seg, 16]  running sum
+    float *po;            // [n_ctas, max_seg, 16, D] unnormalised output
     int32_t *tickets;     // [batch * Hkv]
     int max_seg;
 };
@@ -396,13 +399,24 @@ __host__ __device__ __forceinline__ int64_t stream_cta_of(int64_t items, int64_t
     return ((x + 1) * n - 1) / items;
 }
 
+__device__ __forceinline__ void red_add_shared(float *p, float v) {
+    asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void consumers_sync() {   // the four consumer warps only
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * kStreamConsumers) : "memory");
+}
+
 template <int D, int BLK, int NS>
-__global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_kernel(
+__global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_kernel(
     Prob P, const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __nv_bfloat16 *__restrict__ Q, const int32_t *__restrict__ block_idx, StreamBufs W,
     __nv_bfloat16 *__restrict__ O, float *__restrict__ lse) {
     using SM = StreamSmem<D, BLK, NS>;
     constexpr int DC = SM::DC;
+    constexpr int KW = BLK / kStreamConsumers;   // keys of a block per consumer warp (16 or 32)
+    constexpr int NT = KW / 8;                   // n-tiles of S per warp
+    constexpr int KT = KW / 16;                  // k-steps of P V per warp
     extern __shared__ unsigned char smem_raw[];
     SM &S = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -413,15 +427,21 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_
     const int k_tot = P.k_tot;
     const int64_t bg_first = x0 / k_tot;
     const int nseg = n > 0 ? (int)((x1 - 1) / k_tot - bg_first + 1) : 0;
+    volatile int &fail = S.fail;
 
+    if (warp == kStreamConsumers && lane == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&S.full[s], 1);
-            mbar_init(&S.empty[s], 1);
+            mbar_init(&S.empty[s], kStreamConsumers);
         }
         S.fail = 0;
         fence_barrier_init();
     }
+    for (int e = tid; e < 16 * (D + 8); e += blockDim.x) (&S.ob[0][0])[e] = 0.f;
     __syncthreads();
 
     if (warp == kStreamConsumers) {
@@ -470,10 +490,11 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_
             }
             if (lane == 0) {
                 const int s = k % NS;
-                if (!mbar_wait(&S.empty[s], ((k / NS) & 1) ^ 1)) S.fail = 1;
+                if (!mbar_wait(&S.empty[s], ((k / NS) & 1) ^ 1)) fail = 1;
                 const int j = S.row[a];
                 S.js[s] = j;
-                if (j >= 0) {
+                if (fail) {
+                } else if (j >= 0) {
                     mbar_arrive_expect_tx(&S.full[s], 2 * DC * SM::KV_CHUNK);
                     const int row0 = (int)(bg * P.Lmax + (int64_t)j * BLK);
 #pragma unroll
@@ -485,14 +506,17 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_
                     mbar_arrive(&S.full[s]);   // nothing to load: the slot is skipped
                 }
             }
-            if (__any_sync(0xffffffffu, S.fail != 0)) break;
+            if (__any_sync(0xffffffffu, fail != 0)) break;
         }
     } else {
         // ------------------------------------------------------------------ consumers
+        // Every consumer warp runs the same sequence of items and flushes (the flush has two
+        // consumer-only barriers), also after a failed wait: it then skips the math, never the
+        // control flow.
+        const int key0 = warp * KW;
         float m_r[2], l_r[2];
         float o[D / 8][4];
         uint32_t qf[D / 16][4];
-        int cur = -1;   // current segment (b, g) - bg_first
         auto reset = [&]() {
             m_r[0] = m_r[1] = -INFINITY;
             l_r[0] = l_r[1] = 0.f;
@@ -500,24 +524,59 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_
             for (int dt = 0; dt < D / 8; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
         };
         auto flush = [&](int seg) {
-            const int64_t slot = ((c * kStreamConsumers + warp) * W.max_seg + seg) * 16;
+            const int r0 = lane >> 2;
             float l0 = l_r[0], l1 = l_r[1];
             l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
             l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
             l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
             l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-            const int r0 = lane >> 2;
             if ((lane & 3) == 0) {
-                W.pm[slot + r0] = m_r[0];
-                W.pm[slot + r0 + 8] = m_r[1];
-                W.pl[slot + r0] = l0;
-                W.pl[slot + r0 + 8] = l1;
+                S.mw[warp][r0] = m_r[0];
+                S.mw[warp][r0 + 8] = m_r[1];
+                S.lw[warp][r0] = l0;
+                S.lw[warp][r0 + 8] = l1;
             }
+            consumers_sync();
+            float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
-            for (int dt = 0; dt < D / 8; ++dt) {
-                const int col = dt * 8 + 2 * (lane & 3);
-                *reinterpret_cast<float2 *>(W.po + (slot + r0) * D + col) = make_float2(o[dt][0], o[dt][1]);
-                *reinterpret_cast<float2 *>(W.po + (slot + r0 + 8) * D + col) = make_float2(o[dt][2], o[dt][3]);
+            for (int w = 0; w < kStreamConsumers; ++w) {
+                M0 = fmaxf(M0, S.mw[w][r0]);
+                M1 = fmaxf(M1, S.mw[w][r0 + 8]);
+            }
+            const float f0 = m_r[0] == -INFINITY ? 0.f : ex2_approx(m_r[0] - M0);
+            const float f1 = m_r[1] == -INFINITY ? 0.f : ex2_approx(m_r[1] - M1);
+            const int64_t slot = ((int64_t)c * W.max_seg + seg) * 16;
+            if (tid < 16) {   // the segment's running max and sum per query row
+                float M = -INFINITY, L = 0.f;
+#pragma unroll
+                for (int w = 0; w < kStreamConsumers; ++w) M = fmaxf(M, S.mw[w][tid]);
+#pragma unroll
+                for (int w = 0; w < kStreamConsumers; ++w)
+                    if (S.mw[w][tid] > -INFINITY) L += S.lw[w][tid] * ex2_approx(S.mw[w][tid] - M);
+                W.pm[slot + tid] = M;
+                W.pl[slot + tid] = L;
+            }
+            if (r0 < P.G) {
+#pragma unroll
+                for (int dt = 0; dt < D / 8; ++dt) {
+                    const int col = dt * 8 + 2 * (lane & 3);
+                    red_add_shared(&S.ob[r0][col], o[dt][0] * f0);
+                    red_add_shared(&S.ob[r0][col + 1], o[dt][1] * f0);
+                }
+            }
+            if (r0 + 8 < P.G) {
+#pragma unroll
+                for (int dt = 0; dt < D / 8; ++dt) {
+                    const int col = dt * 8 + 2 * (lane & 3);
+                    red_add_shared(&S.ob[r0 + 8][col], o[dt][2] * f1);
+                    red_add_shared(&S.ob[r0 + 8][col + 1], o[dt][3] * f1);
+                }
+            }
+            consumers_sync();
+            for (int e = tid * 4; e < P.G * D; e += 32 * kStreamConsumers * 4) {
+                float4 *src = reinterpret_cast<float4 *>(&S.ob[e / D][e % D]);
+                *reinterpret_cast<float4 *>(W.po + slot * D + e) = *src;
+                *src = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         };
         auto load_q = [&](int64_t bg) {
@@ -535,42 +594,42 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_
                 qf[ks][3] = ok1 ? *reinterpret_cast<const uint32_t *>(q1 + col + 8) : 0u;
             }
         };
+        int cur = 0;
         reset();
-        for (int k = warp; k < n; k += kStreamConsumers) {
+        if (n > 0) load_q(bg_first);
+        for (int k = 0; k < n; ++k) {
             const int s = k % NS;
-            if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (k / NS) & 1))) {
-                if (lane == 0) S.fail = 1;
-                break;
-            }
             const int64_t x = x0 + k;
             const int64_t bg = x / k_tot;
             const int seg = (int)(bg - bg_first);
             if (seg != cur) {
-                if (cur >= 0) flush(cur);
-                for (int z = cur + 1; z < seg; ++z) {   // segments this warp never touched
-                    reset();
-                    flush(z);
-                }
+                flush(cur);
                 reset();
                 load_q(bg);
                 cur = seg;
             }
+            bool ok = fail == 0;
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&S.full[s], (k / NS) & 1));
+            if (!ok) {
+                if (lane == 0) fail = 1;
+                continue;
+            }
             const int j = S.js[s];
-            if (j >= 0) {
-                const int b = (int)(bg / P.Hkv);
-                const int64_t pos = (int64_t)P.seqlens[b] - 1;
-                const int64_t i = pos / BLK;
+            const int b = (int)(bg / P.Hkv);
+            const int64_t pos = (int64_t)P.seqlens[b] - 1;
+            const int lim = (j == pos / BLK) ? (int)(pos - (int64_t)j * BLK) : BLK - 1;   // last valid key
+            if (j >= 0 && key0 <= lim) {
                 const uint32_t k_base = smem_u32(S.k[s]), v_base = smem_u32(S.v[s]);
-                float sc[BLK / 8][4];
+                float sc[NT][4];
 #pragma unroll
-                for (int nt = 0; nt < BLK / 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+                for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const int cch = ks / 4;
 #pragma unroll
-                    for (int nt = 0; nt < BLK / 8; nt += 2) {
+                    for (int nt = 0; nt < NT; nt += 2) {
                         const int mi = lane >> 3;
-                        const int key = (nt + (mi >> 1)) * 8 + (lane & 7);
+                        const int key = key0 + (nt + (mi >> 1)) * 8 + (lane & 7);
                         const int ch = (ks * 2 + (mi & 1)) & 7;
                         uint32_t b0, b1, b2, b3;
                         ldsm_x4(k_base + cch * SM::KV_CHUNK + sw128(key, ch), b0, b1, b2, b3);
@@ -578,32 +637,32 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_
                         mma_bf16_16816(sc[nt + 1], qf[ks], b2, b3);
                     }
                 }
-                const int lim = (j == i) ? (int)(pos - (int64_t)j * BLK) : BLK - 1;
                 float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-                for (int nt = 0; nt < BLK / 8; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int key = nt * 8 + 2 * (lane & 3) + (e & 1);
+                        const int key = key0 + nt * 8 + 2 * (lane & 3) + (e & 1);
                         const float t = key <= lim ? sc[nt][e] * P.scale_log2 : -INFINITY;
                         sc[nt][e] = t;
                         mx[e >> 1] = fmaxf(mx[e >> 1], t);
                     }
-                float alpha[2];
+                float alpha[2], m_use[2];
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr) {
                     mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
                     mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
                     const float m_new = fmaxf(m_r[rr], mx[rr]);
-                    alpha[rr] = ex2_approx(m_r[rr] - m_new);
+                    m_use[rr] = m_new == -INFINITY ? 0.f : m_new;   // a row with no valid key yet
+                    alpha[rr] = ex2_approx(m_r[rr] - m_use[rr]);
                     m_r[rr] = m_new;
                 }
                 float ls[2] = {0.f, 0.f};
 #pragma unroll
-                for (int nt = 0; nt < BLK / 8; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float p = ex2_approx(sc[nt][e] - m_r[e >> 1]);
+                        const float p = ex2_approx(sc[nt][e] - m_use[e >> 1]);
                         sc[nt][e] = p;
                         ls[e >> 1] += p;
                     }
@@ -617,7 +676,7 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_
                     o[dt][3] *= alpha[1];
                 }
 #pragma unroll
-                for (int kt = 0; kt < BLK / 16; ++kt) {
+                for (int kt = 0; kt < KT; ++kt) {
                     uint32_t pa[4];
                     pa[0] = pack_bf16(sc[2 * kt][0], sc[2 * kt][1]);
                     pa[1] = pack_bf16(sc[2 * kt][2], sc[2 * kt][3]);
@@ -626,7 +685,7 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_
 #pragma unroll
                     for (int dt = 0; dt < D / 8; dt += 2) {
                         const int mi = lane >> 3;
-                        const int key = kt * 16 + (mi & 1) * 8 + (lane & 7);
+                        const int key = key0 + kt * 16 + (mi & 1) * 8 + (lane & 7);
                         const int dch = dt + (mi >> 1);
                         uint32_t b0, b1, b2, b3;
                         ldsm_x4_t(v_base + (dch >> 3) * SM::KV_CHUNK + sw128(key, dch & 7), b0, b1, b2, b3);
@@ -638,63 +697,159 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 1) decode_stream_
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.empty[s]);
         }
-        if (cur >= 0) flush(cur);
-        for (int z = cur + 1; z < nseg; ++z) {
-            reset();
-            flush(z);
-        }
+        if (n > 0) flush(cur);
     }
 
-    // every partial of this CTA is written: take the tickets of its segments; the CTA that
-    // completes a segment merges it
+    // every partial of this CTA is written: take the tickets of its segments (up to 32 at a time,
+    // in parallel); the CTA that completes a segment merges it.  The merge issues its global loads
+    // in two rounds (the partials' maxima and sums, then their O rows), chunks of kPC partials at
+    // a time.  Shared memory reused (the loop is over): S.row -> slot of each partial, S.mw[0] /
+    // S.lw[0] -> the segment's running max and sum per row, S.ob -> per chunk the partials' maxima
+    // (then weights 2^(m_p - m) / l) and sums.
     __threadfence();
     __syncthreads();
-    for (int seg = 0; seg < nseg; ++seg) {
-        const int64_t bg = bg_first + seg;
-        const int64_t c_first = stream_cta_of(items, bg * k_tot, nc);
-        const int64_t c_last = stream_cta_of(items, (bg + 1) * k_tot - 1, nc);
-        if (tid == 0) S.last = atomicAdd(&W.tickets[bg], 1) == (int)(c_last - c_first);
+    constexpr int kPC = 32;
+    constexpr int kThreads = 32 * (kStreamConsumers + 1);
+    constexpr int kAcc = (16 * D / 4 + kThreads - 1) / kThreads;
+    static_assert(2 * kPC * 16 <= 16 * (D + 8), "merge chunk must fit the flush buffer");
+    int *slot_of = S.row;
+    float *pm_s = &S.ob[0][0];
+    float *pl_s = pm_s + kPC * 16;
+    const int G = P.G;
+    for (int s0 = 0; s0 < nseg; s0 += 32) {
+        if (tid < min(32, nseg - s0)) {
+            const int64_t bg = bg_first + s0 + tid;
+            const int64_t c_first = stream_cta_of(items, bg * k_tot, nc);
+            const int64_t c_last = stream_cta_of(items, (bg + 1) * k_tot - 1, nc);
+            S.lastf[tid] = atomicAdd(&W.tickets[bg], 1) == (int)(c_last - c_first);
+        }
         __syncthreads();
-        if (S.last) {
+        for (int seg = s0; seg < min(nseg, s0 + 32); ++seg) {
+            if (!S.lastf[seg - s0]) continue;   // uniform across the CTA
             __threadfence();
-            const int b = (int)(bg / P.Hkv), g = (int)(bg % P.Hkv);
-            for (int e = tid; e < P.G * D; e += blockDim.x) {
-                const int r = e / D, col = e % D;
-                float M = -INFINITY;
-                for (int64_t cc = c_first; cc <= c_last; ++cc) {
-                    const int sg = (int)(bg - stream_begin(items, cc, nc) / k_tot);
-                    for (int w = 0; w < kStreamConsumers; ++w)
-                        M = fmaxf(M, __ldcg(&W.pm[((cc * kStreamConsumers + w) * W.max_seg + sg) * 16 + r]));
+            const int64_t bg = bg_first + seg;
+            const int64_t c_first = stream_cta_of(items, bg * k_tot, nc);
+            const int np = (int)(stream_cta_of(items, (bg + 1) * k_tot - 1, nc) - c_first + 1);
+            for (int p = tid; p < np; p += kThreads) {
+                const int64_t cc = c_first + p;
+                slot_of[p] = (int)((cc * W.max_seg + (bg - stream_begin(items, cc, nc) / k_tot)) * 16);
+            }
+            if (tid < G) {
+                S.mw[0][tid] = -INFINITY;
+                S.lw[0][tid] = 0.f;
+            }
+            // round 1: running max and sum over the partials, chunk by chunk
+            for (int c0 = 0; c0 < np; c0 += kPC) {
+                const int cn = min(kPC, np - c0);
+                __syncthreads();
+                for (int e = tid; e < cn * G; e += kThreads) {
+                    const int q = e / G, r = e % G;
+                    const int sl = slot_of[c0 + q] + r;
+                    pm_s[q * 16 + r] = __ldcg(&W.pm[sl]);
+                    pl_s[q * 16 + r] = __ldcg(&W.pl[sl]);
                 }
-                float L = 0.f, acc = 0.f;
-                if (M > -INFINITY) {
-                    for (int64_t cc = c_first; cc <= c_last; ++cc) {
-                        const int sg = (int)(bg - stream_begin(items, cc, nc) / k_tot);
-                        for (int w = 0; w < kStreamConsumers; ++w) {
-                            const int64_t sl = ((cc * kStreamConsumers + w) * W.max_seg + sg) * 16 + r;
-                            const float mm = __ldcg(&W.pm[sl]);
-                            if (mm == -INFINITY) continue;
-                            const float f = ex2_approx(mm - M);
-                            L += __ldcg(&W.pl[sl]) * f;
-                            acc += __ldcg(&W.po[sl * D + col]) * f;
+                __syncthreads();
+                if (tid < G) {
+                    float M = S.mw[0][tid], L = S.lw[0][tid];
+                    float cm = -INFINITY;
+                    for (int q = 0; q < cn; ++q) cm = fmaxf(cm, pm_s[q * 16 + tid]);
+                    if (cm > -INFINITY) {
+                        const float Mn = fmaxf(M, cm);
+                        L = (M > -INFINITY) ? L * ex2_approx(M - Mn) : 0.f;
+                        for (int q = 0; q < cn; ++q) {
+                            const float mm = pm_s[q * 16 + tid];
+                            if (mm > -INFINITY) L += pl_s[q * 16 + tid] * ex2_approx(mm - Mn);
+                        }
+                        M = Mn;
+                    }
+                    S.mw[0][tid] = M;
+                    S.lw[0][tid] = L;
+                }
+            }
+            // round 2: O = sum_p w_p O_p, w_p = 2^(m_p - m) / l
+            float4 acc[kAcc];
+#pragma unroll
+            for (int u = 0; u < kAcc; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int c0 = 0; c0 < np; c0 += kPC) {
+                const int cn = min(kPC, np - c0);
+                __syncthreads();
+                if (np > kPC) {   // segments over more than kPC CTAs: reload this chunk's maxima
+                    for (int e = tid; e < cn * G; e += kThreads) {
+                        const int q = e / G, r = e % G;
+                        pm_s[q * 16 + r] = __ldcg(&W.pm[slot_of[c0 + q] + r]);
+                    }
+                    __syncthreads();
+                }
+                if (tid < G) {
+                    const float M = S.mw[0][tid], L = S.lw[0][tid];
+                    for (int q = 0; q < cn; ++q) {
+                        const float mm = pm_s[q * 16 + tid];
+                        pm_s[q * 16 + tid] = (mm > -INFINITY && L > 0.f) ? ex2_approx(mm - M) / L : 0.f;
+                    }
+                }
+                __syncthreads();
+                for (int q0 = 0; q0 < cn; q0 += 4) {
+                    float4 v[kAcc][4];
+#pragma unroll
+                    for (int u = 0; u < kAcc; ++u) {
+                        const int e4 = tid + u * kThreads;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            v[u][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (e4 * 4 < G * D && q0 + q < cn) {
+                                const int r = (e4 * 4) / D, col = (e4 * 4) % D;
+                                v[u][q] = __ldcg(reinterpret_cast<const float4 *>(
+                                    W.po + (int64_t)(slot_of[c0 + q0 + q] + r) * D + col));
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < kAcc; ++u) {
+                        const int e4 = tid + u * kThreads;
+                        if (e4 * 4 < G * D) {
+                            const int r = (e4 * 4) / D;
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float wv = q0 + q < cn ? pm_s[(q0 + q) * 16 + r] : 0.f;
+                                acc[u].x += wv * v[u][q].x;
+                                acc[u].y += wv * v[u][q].y;
+                                acc[u].z += wv * v[u][q].z;
+                                acc[u].w += wv * v[u][q].w;
+                            }
                         }
                     }
                 }
-                const int64_t orow = (int64_t)b * P.Hq + (int64_t)g * P.G + r;
-                O[orow * D + col] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
-                if (lse && col == 0) lse[orow] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+            }
+            const int b = (int)(bg / P.Hkv), g = (int)(bg % P.Hkv);
+#pragma unroll
+            for (int u = 0; u < kAcc; ++u) {
+                const int e4 = tid + u * kThreads;
+                if (e4 * 4 < G * D) {
+                    const int r = (e4 * 4) / D, col = (e4 * 4) % D;
+                    const int64_t orow = (int64_t)b * P.Hq + (int64_t)g * G + r;
+                    uint2 pk;
+                    pk.x = pack_bf16(acc[u].x, acc[u].y);
+                    pk.y = pack_bf16(acc[u].z, acc[u].w);
+                    *reinterpret_cast<uint2 *>(O + orow * D + col) = pk;
+                    if (lse && col == 0) {
+                        const float M = S.mw[0][r], L = S.lw[0][r];
+                        lse[orow] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+                    }
+                }
             }
             if (tid == 0) W.tickets[bg] = 0;
+            __syncthreads();   // shared scratch free for the next segment
         }
-        __syncthreads();
+        __syncthreads();       // lastf free for the next group
     }
     if (S.fail && tid == 0) report(P.err, kErrTimeout);
 }
 
 template <int D, int BLK>
 struct StreamCfg {
-    // a multiple of the consumer count: two stages per consumer warp where 32 KB blocks allow it
-    static constexpr int NS = (2 * D * BLK * 2 <= 32768) ? 2 * kStreamConsumers : kStreamConsumers;
+    // about 96 KB of K/V in flight per CTA, two CTAs per SM where the stages allow
+    static constexpr int STAGE = 2 * D * BLK * 2;
+    static constexpr int NS = STAGE <= 16384 ? 6 : 3;
     static size_t smem() { return sizeof(StreamSmem<D, BLK, NS>) + 1024; }
 };
 
@@ -705,9 +860,8 @@ void decode_stream_geometry(const Prob &P, int num_sms, int &n_ctas, int &max_se
     else if (P.D == 128 && P.B == 128) smem = StreamCfg<128, 128>::smem();
     else if (P.D == 64 && P.B == 64) smem = StreamCfg<64, 64>::smem();
     else smem = StreamCfg<64, 128>::smem();
-    const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(2, (size_t)(227 * 1024) / smem));
-    static_assert(StreamCfg<128, 64>::NS % kStreamConsumers == 0 && StreamCfg<128, 128>::NS % kStreamConsumers == 0,
-                  "stage count must be a multiple of the consumer warps");
+    // the SM's 228 KB of shared memory less 1 KB reserved per resident CTA
+    const int per_sm = smem + 1024 <= (size_t)114 * 1024 ? 2 : 1;
     const int64_t items = (int64_t)P.batch * P.Hkv * P.k_tot;
     n_ctas = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms * per_sm, items));
     const int64_t per_cta = ceil_div<int64_t>(items, n_ctas);
@@ -718,7 +872,7 @@ size_t decode_stream_ws_bytes(const Prob &P, int num_sms) {
     int n_ctas, max_seg;
     decode_stream_geometry(P, num_sms, n_ctas, max_seg);
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
-    const size_t rows = (size_t)n_ctas * kStreamConsumers * max_seg * 16;
+    const size_t rows = (size_t)n_ctas * max_seg * 16;
     return 2 * a(sizeof(float) * rows) + a(sizeof(float) * rows * P.D) + a(sizeof(int32_t) * P.batch * P.Hkv);
 }
 
@@ -742,7 +896,7 @@ cudaError_t launch_decode_stream(const Prob &P, const CUtensorMap &tk, const CUt
     int n_ctas, max_seg;
     decode_stream_geometry(P, num_sms, n_ctas, max_seg);
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
-    const size_t rows = (size_t)n_ctas * kStreamConsumers * max_seg * 16;
+    const size_t rows = (size_t)n_ctas * max_seg * 16;
     char *base = static_cast<char *>(ws);
     StreamBufs W;
     W.pm = reinterpret_cast<float *>(base);

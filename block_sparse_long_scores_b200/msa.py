@@ -187,7 +187,7 @@ def msa_sparse_attn_decode(cfg: Config, shape: Shape, q, k_cache, v_cache, block
 def msa_sparse_attn_decode_noalloc(cfg: Config, shape: Shape, q, k_cache, v_cache, block_idx, o, lse,
                                    err_flag=None, stream=None):
     """msa_sparse_attn_decode without a workspace argument, for callers that cannot allocate:
-    scratch comes from the library's fixed 40 MiB device array (see include/msa.h for the limit,
+    scratch comes from the library's fixed 40 MiB device array (include/msa.h gives the limit,
     the first-call set-up and why overlapping calls must be serialised)."""
     rc = lib().msa_sparse_attn_decode_noalloc(ctypes.byref(cfg), ctypes.byref(shape), _ptr(q), _ptr(k_cache),
                                               _ptr(v_cache), _ptr(block_idx), _ptr(o), _ptr(lse), _ptr(err_flag),

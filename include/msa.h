@@ -205,10 +205,10 @@ msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *
  * a fixed 40 MiB array in device global memory that the library declares; it calls no
  * cudaMalloc, cudaFree or other allocating routine.
  *  - Limit: a problem whose split partials need more than 40 MiB returns MSA_ERR_WORKSPACE and
- *    launches nothing.  The partials take about n_cta x 3 x (ceil(batch x Hkv x k_tot / n_cta /
- *    k_tot) + 1) x 16 x (head_dim + 2) x 4 bytes, n_cta = the GPU's SM count (148 on B200; twice
- *    that for head_dim 64 with 64-token blocks): 7 MiB for both decode workloads of this
- *    repository; with 4 kv heads and 66 selected blocks, batches up to about 370 sequences fit.
+ *    launches nothing.  The partials take about n_cta x (ceil(batch x Hkv x k_tot / n_cta / k_tot)
+ *    + 1) x 16 x (head_dim + 2) x 4 bytes, n_cta = 2 x the GPU's SM count (296 on B200; 1 x for
+ *    head_dim 128 with 128-token blocks): 4.7 MiB for both decode workloads of this repository;
+ *    with 4 kv heads and 66 selected blocks, batches up to about 1,100 sequences fit.
  *  - Set-up: the first call on a device looks up the array's device address (with that device
  *    current) and caches it; make that first call before any CUDA stream capture.
  *  - Sharing: every call on a device uses the same array, and the array keeps the last call's

@@ -229,6 +229,23 @@ def test_decode_small_ragged():
     _decode_check(w, x)
 
 
+def test_decode_many_short_sequences():
+    # 300 sequences: every CTA of the streaming grid covers several (sequence, kv head) segments,
+    # so in-CTA flushes and cross-CTA merges both run many times
+    lens = tuple(int(v) for v in np.random.default_rng(21).integers(1, 2049, size=300))
+    w = scaled_down(WORKLOADS["decode_128k"], lens)
+    x = make_inputs(w, device=DEV, seed=21)
+    _decode_check(w, x)
+
+
+def test_decode_single_sequence():
+    # one sequence: every CTA holds one or two selected blocks, so a segment's merge spans more
+    # partials than one merge chunk
+    w = scaled_down(WORKLOADS["decode_128k"], (5000,))
+    x = make_inputs(w, device=DEV, seed=22)
+    _decode_check(w, x)
+
+
 def test_decode_ragged_shape_with_ties():
     w = scaled_down(WORKLOADS["ragged_decode"], (129, 5000, 1, 3000))
     x = make_inputs(w, device=DEV, seed=9)

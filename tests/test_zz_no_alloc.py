@@ -58,12 +58,13 @@ def test_noalloc_decode_second_problem_after_first():
 
 
 def test_noalloc_decode_rejects_problems_beyond_its_scratch():
-    # 1024 short sequences x 4 kv heads x 66 slots make ~145 MiB of split partials: refused before
+    # 4096 short sequences x 4 kv heads x 66 slots make ~140 MiB of split partials: refused before
     # any pointer is used, nothing launched
-    w = WORKLOADS["decode_128k"].with_(seqlens=(64,) * 1024)
+    nseq = 4096
+    w = WORKLOADS["decode_128k"].with_(seqlens=(64,) * nseq)
     cfg = msa.make_config(w.Hq, w.Hkv, w.D, w.B, w.d, w.n_topk, w.use_sink)
-    seqlens = torch.full((1024,), 64, dtype=torch.int32, device="cuda")
-    shape = msa.decode_shape(seqlens, 1024, 64, w.B)
+    seqlens = torch.full((nseq,), 64, dtype=torch.int32, device="cuda")
+    shape = msa.decode_shape(seqlens, nseq, 64, w.B)
     fake = torch.empty(16, dtype=torch.uint8, device="cuda")
     with pytest.raises(msa.MSAError) as ei:
         msa.msa_sparse_attn_decode_noalloc(cfg, shape, fake, fake, fake, fake, fake, None)
