@@ -442,7 +442,7 @@ msa_status_t msa_sparse_attn_decode_noalloc(const msa_config_t *cfg, const msa_s
     if (!scratch) return MSA_ERR_CUDA;
     CUtensorMap tq, tk, tv;
     if (!decode_maps(P, q, k_cache, v_cache, &tq, &tk, &tv)) return MSA_ERR_CUDA;
-    // the launcher clears the merge tickets in the scratch before its kernel runs
+    // the scratch needs no clearing: its merge counters are tagged with a per-call generation
     cudaError_t e = launch_decode_stream(P, tk, tv, q, block_idx, o, lse, scratch, num_sms(),
                                          static_cast<cudaStream_t>(stream));
     return cuda_status(e, 1);

@@ -15,6 +15,8 @@
 // (scores are kept in log2 units: t = scale * log2(e) * q.k).
 #include <algorithm>
 
+#include <atomic>
+
 #include "launch.cuh"
 
 namespace msa {
@@ -386,21 +388,32 @@ struct StreamSmem {
 };
 
 struct StreamBufs {
-    float *pm;            // [n_ctas, max_seg, 16]  running max (log2 units)
-    float *pl;            // [n_ctas, max_seg, 16]  running sum
-    float *po;            // [n_ctas, max_seg, 16, D] unnormalised output
-    int32_t *tickets;     // [batch * Hkv]
+    float *pm;                      // [n_ctas, max_seg, 16]  running max (log2 units)
+    float *pl;                      // [n_ctas, max_seg, 16]  running sum
+    float *po;                      // [n_ctas, max_seg, 16, D] unnormalised output
+    unsigned long long *tickets;    // [batch * Hkv]: (call generation << 32) | partials merged
     int max_seg;
+    uint32_t gen;                   // this call's generation (never 0)
 };
+
+// Take a segment's ticket: a count tagged with the call's generation, so that a count left by an
+// earlier call (or anything else in a fresh workspace) reads as zero and needs no clearing.
+// Returns the number of partials counted before this one.
+__device__ __forceinline__ uint32_t take_ticket(unsigned long long *t, uint32_t gen) {
+    unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(t);
+    while (true) {
+        const uint32_t n = (uint32_t)(cur >> 32) == gen ? (uint32_t)cur : 0u;
+        const unsigned long long want = ((unsigned long long)gen << 32) | (n + 1u);
+        const unsigned long long seen = atomicCAS(t, cur, want);
+        if (seen == cur) return n;
+        cur = seen;
+    }
+}
 
 __host__ __device__ __forceinline__ int64_t stream_begin(int64_t items, int64_t c, int64_t n) { return items * c / n; }
 // CTA whose range holds item x (largest c with stream_begin(c) <= x)
 __host__ __device__ __forceinline__ int64_t stream_cta_of(int64_t items, int64_t x, int64_t n) {
     return ((x + 1) * n - 1) / items;
-}
-
-__device__ __forceinline__ void red_add_shared(float *p, float v) {
-    asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ void consumers_sync() {   // the four consumer warps only
@@ -443,6 +456,8 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
     }
     for (int e = tid; e < 16 * (D + 8); e += blockDim.x) (&S.ob[0][0])[e] = 0.f;
     __syncthreads();
+    griddep_wait();     // block lists, queries and lengths may come from the previous kernel
+    griddep_launch();
 
     if (warp == kStreamConsumers) {
         // ------------------------------------------------------------------ producer (warp)
@@ -556,27 +571,32 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                 W.pm[slot + tid] = M;
                 W.pl[slot + tid] = L;
             }
-            if (r0 < P.G) {
+            // warps add their rows in a fixed order (warp 0 stores, then 1, 2, 3 add), so the
+            // partial does not depend on timing
+#pragma unroll 1
+            for (int w = 0; w < kStreamConsumers; ++w) {
+                if (w > 0) consumers_sync();
+                if (warp != w) continue;
 #pragma unroll
                 for (int dt = 0; dt < D / 8; ++dt) {
                     const int col = dt * 8 + 2 * (lane & 3);
-                    red_add_shared(&S.ob[r0][col], o[dt][0] * f0);
-                    red_add_shared(&S.ob[r0][col + 1], o[dt][1] * f0);
-                }
-            }
-            if (r0 + 8 < P.G) {
-#pragma unroll
-                for (int dt = 0; dt < D / 8; ++dt) {
-                    const int col = dt * 8 + 2 * (lane & 3);
-                    red_add_shared(&S.ob[r0 + 8][col], o[dt][2] * f1);
-                    red_add_shared(&S.ob[r0 + 8][col + 1], o[dt][3] * f1);
+                    float2 *a = reinterpret_cast<float2 *>(&S.ob[r0][col]);
+                    float2 *c = reinterpret_cast<float2 *>(&S.ob[r0 + 8][col]);
+                    const float2 va = make_float2(o[dt][0] * f0, o[dt][1] * f0);
+                    const float2 vc = make_float2(o[dt][2] * f1, o[dt][3] * f1);
+                    if (w == 0) {
+                        if (r0 < P.G) *a = va;
+                        if (r0 + 8 < P.G) *c = vc;
+                    } else {
+                        if (r0 < P.G) *a = make_float2(a->x + va.x, a->y + va.y);
+                        if (r0 + 8 < P.G) *c = make_float2(c->x + vc.x, c->y + vc.y);
+                    }
                 }
             }
             consumers_sync();
             for (int e = tid * 4; e < P.G * D; e += 32 * kStreamConsumers * 4) {
-                float4 *src = reinterpret_cast<float4 *>(&S.ob[e / D][e % D]);
-                *reinterpret_cast<float4 *>(W.po + slot * D + e) = *src;
-                *src = make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4 *>(W.po + slot * D + e) =
+                    *reinterpret_cast<const float4 *>(&S.ob[e / D][e % D]);
             }
         };
         auto load_q = [&](int64_t bg) {
@@ -721,7 +741,7 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
             const int64_t bg = bg_first + s0 + tid;
             const int64_t c_first = stream_cta_of(items, bg * k_tot, nc);
             const int64_t c_last = stream_cta_of(items, (bg + 1) * k_tot - 1, nc);
-            S.lastf[tid] = atomicAdd(&W.tickets[bg], 1) == (int)(c_last - c_first);
+            S.lastf[tid] = take_ticket(&W.tickets[bg], W.gen) == (uint32_t)(c_last - c_first);
         }
         __syncthreads();
         for (int seg = s0; seg < min(nseg, s0 + 32); ++seg) {
@@ -837,7 +857,6 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                     }
                 }
             }
-            if (tid == 0) W.tickets[bg] = 0;
             __syncthreads();   // shared scratch free for the next segment
         }
         __syncthreads();       // lastf free for the next group
@@ -873,7 +892,8 @@ size_t decode_stream_ws_bytes(const Prob &P, int num_sms) {
     decode_stream_geometry(P, num_sms, n_ctas, max_seg);
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
     const size_t rows = (size_t)n_ctas * max_seg * 16;
-    return 2 * a(sizeof(float) * rows) + a(sizeof(float) * rows * P.D) + a(sizeof(int32_t) * P.batch * P.Hkv);
+    return 2 * a(sizeof(float) * rows) + a(sizeof(float) * rows * P.D) +
+           a(sizeof(unsigned long long) * P.batch * P.Hkv);
 }
 
 template <int D, int BLK>
@@ -885,9 +905,8 @@ static cudaError_t launch_stream_t(const Prob &P, const CUtensorMap &tk, const C
     auto kern = decode_stream_kernel<D, BLK, NS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<n_ctas, 32 * (kStreamConsumers + 1), smem, st>>>(P, tk, tv, (const __nv_bfloat16 *)q, block_idx, W,
-                                                           (__nv_bfloat16 *)O, lse);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(n_ctas), dim3(32 * (kStreamConsumers + 1)), smem, st, P, tk, tv,
+                      (const __nv_bfloat16 *)q, block_idx, W, (__nv_bfloat16 *)O, lse);
 }
 
 cudaError_t launch_decode_stream(const Prob &P, const CUtensorMap &tk, const CUtensorMap &tv, const void *q,
@@ -902,10 +921,13 @@ cudaError_t launch_decode_stream(const Prob &P, const CUtensorMap &tk, const CUt
     W.pm = reinterpret_cast<float *>(base);
     W.pl = reinterpret_cast<float *>(base + a(sizeof(float) * rows));
     W.po = reinterpret_cast<float *>(base + 2 * a(sizeof(float) * rows));
-    W.tickets = reinterpret_cast<int32_t *>(base + 2 * a(sizeof(float) * rows) + a(sizeof(float) * rows * P.D));
+    W.tickets = reinterpret_cast<unsigned long long *>(base + 2 * a(sizeof(float) * rows) +
+                                                       a(sizeof(float) * rows * P.D));
     W.max_seg = max_seg;
-    cudaError_t e = cudaMemsetAsync(W.tickets, 0, sizeof(int32_t) * P.batch * P.Hkv, st);
-    if (e != cudaSuccess) return e;
+    static std::atomic<uint32_t> generation{0};
+    uint32_t gen;
+    do gen = ++generation; while (gen == 0);
+    W.gen = gen;
     ProfScope prof("decode_attn", st);
     if (P.D == 128 && P.B == 64) return launch_stream_t<128, 64>(P, tk, tv, q, block_idx, W, n_ctas, O, lse, st);
     if (P.D == 128 && P.B == 128) return launch_stream_t<128, 128>(P, tk, tv, q, block_idx, W, n_ctas, O, lse, st);

@@ -9,7 +9,8 @@
 // index queries on the CUDA cores straight into a 128-byte-swizzled smem tile (the UMMA A
 // operand), then sweeps the sequence's block keys 128 at a time (TMA -> smem B operand ->
 // tcgen05.mma, fp32 accumulator in TMEM -> registers -> global).  Decode rows (one token per
-// sequence, each against its own cache of block keys) are a batched GEMV on the CUDA cores.
+// sequence, each against its own cache of block keys) are a batched GEMV on the CUDA cores, bound
+// by the bandwidth of reading the block keys.
 #include "launch.cuh"
 
 namespace msa {
@@ -273,53 +274,88 @@ __global__ void __launch_bounds__(128) index_scores_tc_kernel(Prob P, const __gr
 
 // ------------------------------------------------------------------- decode scores (GEMV)
 
-// grid (ceil(max_blocks / 256), Hkv, rows); 256 threads; one block key per thread.
+// grid (ceil(max_blocks / 256), Hkv, rows); 256 threads; 256 block keys per CTA.
+// The block keys' loads are issued first; while they are in flight the CTA stages W_q in shared
+// memory and rebuilds the index query (64 outputs x 4 parts of D/4 terms).  Block keys stream coalesced: 8 lanes share one
+// 128-byte key (16 bytes each, 8 of the 64 index dims), so a warp instruction reads 512
+// contiguous bytes; the 8 partial dot products are summed with three shuffles.
+constexpr int kDecKeysPerCta = 256;
+
 template <int D>
-__global__ void __launch_bounds__(256) index_scores_decode_kernel(Prob P, const __nv_bfloat16 *__restrict__ Q,
+__global__ void __launch_bounds__(256, 4) index_scores_decode_kernel(Prob P, const __nv_bfloat16 *__restrict__ Q,
                                                                   const __nv_bfloat16 *__restrict__ Wq,
                                                                   const __nv_bfloat16 *__restrict__ kidx,
                                                                   float *__restrict__ scores, int64_t stride,
                                                                   __nv_bfloat16 *__restrict__ qidx_out) {
+    constexpr int EP = D / 4;                       // W_q rows per part
+    constexpr int IT = kDecKeysPerCta / 32;         // keys per 8-lane group
+    __shared__ __align__(16) __nv_bfloat16 wq_s[D * 64];
     __shared__ float qbar[D];
+    __shared__ float qpart[4][64];
     __shared__ float qi[64];
-    const int tid = threadIdx.x, g = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = blockIdx.y;
+    griddep_wait();
+    griddep_launch();
     const int64_t r = P.row_begin + blockIdx.z;
     const int b = (int)r;
-    const int64_t len = P.seqlens[b];
-    const int64_t i = (len - 1) / P.B;
-    const int64_t j0 = (int64_t)blockIdx.x * 256;
-    if (j0 >= i && !(blockIdx.x == 0 && qidx_out)) return;
+    const int64_t i = ((int64_t)P.seqlens[b] - 1) / P.B;
+    const int64_t j0 = (int64_t)blockIdx.x * kDecKeysPerCta;
+    const bool write_q = blockIdx.x == 0 && qidx_out;
+    if (j0 >= i && !write_q) return;
 
-    for (int e = tid; e < D; e += blockDim.x) {
+    // the block keys do not depend on the index query: their loads go out first and land while
+    // the query is built
+    const int64_t jhi = lmin(j0 + kDecKeysPerCta, i);   // candidates are [use_sink, i)
+    const int chunk = lane & 7;
+    const __nv_bfloat16 *base = kidx + ((int64_t)b * P.Hkv + g) * P.max_blocks * 64;
+    uint4 raw[IT];
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+        const int64_t j = j0 + it * 32 + warp * 4 + (lane >> 3);
+        raw[it] = j < jhi ? reinterpret_cast<const uint4 *>(base + j * 64)[chunk] : make_uint4(0u, 0u, 0u, 0u);
+    }
+
+    const int o = tid & 63, part = tid >> 6;
+#pragma unroll
+    for (int c = tid; c < D * 64 / 8; c += 256)
+        reinterpret_cast<uint4 *>(wq_s)[c] = reinterpret_cast<const uint4 *>(Wq)[c];
+    if (tid < D) {
         float acc = 0.f;
-        for (int h = 0; h < P.G; ++h) acc += __bfloat162float(Q[(r * P.Hq + (int64_t)g * P.G + h) * D + e]);
-        qbar[e] = acc / (float)P.G;
+        for (int h = 0; h < P.G; ++h) acc += __bfloat162float(Q[(r * P.Hq + (int64_t)g * P.G + h) * D + tid]);
+        qbar[tid] = acc / (float)P.G;
     }
     __syncthreads();
-    if (tid < 64) {
-        float acc = 0.f;
-        for (int e = 0; e < D; ++e) acc = fmaf(qbar[e], __bfloat162float(Wq[e * 64 + tid]), acc);
-        const __nv_bfloat16 hb = __float2bfloat16_rn(acc);
-        qi[tid] = __bfloat162float(hb);
-        if (blockIdx.x == 0 && qidx_out) qidx_out[((r - P.row_begin) * P.Hkv + g) * 64 + tid] = hb;
-    }
-    __syncthreads();
-    const int64_t j = j0 + tid;
-    if (j < P.use_sink || j >= i) return;
-    const __nv_bfloat16 *kr = kidx + (((int64_t)b * P.Hkv + g) * P.max_blocks + j) * 64;
     float acc = 0.f;
 #pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-        uint4 raw = reinterpret_cast<const uint4 *>(kr)[c8];
-        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+    for (int k = 0; k < EP; ++k) acc = fmaf(qbar[part * EP + k], __bfloat162float(wq_s[(part * EP + k) * 64 + o]), acc);
+    qpart[part][o] = acc;
+    __syncthreads();
+    if (tid < 64) {
+        const __nv_bfloat16 hb = __float2bfloat16_rn((qpart[0][tid] + qpart[1][tid]) + (qpart[2][tid] + qpart[3][tid]));
+        qi[tid] = __bfloat162float(hb);
+        if (write_q) qidx_out[((r - P.row_begin) * P.Hkv + g) * 64 + tid] = hb;
+    }
+    __syncthreads();
+    float q8[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) q8[t] = qi[chunk * 8 + t];
+    float *srow = scores + ((r - P.row_begin) * P.Hkv + g) * stride;
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[it]);
+        float part_dot = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            float2 f = __bfloat1622float2(h2[q]);
-            acc = fmaf(qi[c8 * 8 + 2 * q], f.x, acc);
-            acc = fmaf(qi[c8 * 8 + 2 * q + 1], f.y, acc);
+            const float2 f = __bfloat1622float2(h2[q]);
+            part_dot = fmaf(q8[2 * q], f.x, part_dot);
+            part_dot = fmaf(q8[2 * q + 1], f.y, part_dot);
         }
+        part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 1);
+        part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 2);
+        part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 4);
+        const int64_t j = j0 + it * 32 + warp * 4 + (lane >> 3);
+        if (chunk == 0 && j >= P.use_sink && j < jhi) srow[j] = part_dot;
     }
-    scores[((r - P.row_begin) * P.Hkv + g) * stride + j] = acc;
 }
 
 // ------------------------------------------------------------------------------ launchers
@@ -369,17 +405,15 @@ cudaError_t launch_index_scores_decode(const Prob &P, const void *Q, const void 
                                        int64_t stride, void *qidx_out, cudaStream_t st) {
     const int64_t rows = P.row_end - P.row_begin;
     if (rows <= 0) return cudaSuccess;
-    dim3 grid((unsigned)ceil_div<int64_t>(P.max_blocks, 256), (unsigned)P.Hkv, (unsigned)rows);
+    dim3 grid((unsigned)ceil_div<int64_t>(P.max_blocks, kDecKeysPerCta), (unsigned)P.Hkv, (unsigned)rows);
     ProfScope prof("index_scores", st);
     if (P.D == 128)
-        index_scores_decode_kernel<128><<<grid, 256, 0, st>>>(P, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)Wq,
-                                                              (const __nv_bfloat16 *)kidx, scores, stride,
-                                                              (__nv_bfloat16 *)qidx_out);
-    else
-        index_scores_decode_kernel<64><<<grid, 256, 0, st>>>(P, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)Wq,
-                                                             (const __nv_bfloat16 *)kidx, scores, stride,
-                                                             (__nv_bfloat16 *)qidx_out);
-    return cudaGetLastError();
+        return launch_pdl(index_scores_decode_kernel<128>, grid, dim3(256), 0, st, P, (const __nv_bfloat16 *)Q,
+                          (const __nv_bfloat16 *)Wq, (const __nv_bfloat16 *)kidx, scores, stride,
+                          (__nv_bfloat16 *)qidx_out);
+    return launch_pdl(index_scores_decode_kernel<64>, grid, dim3(256), 0, st, P, (const __nv_bfloat16 *)Q,
+                      (const __nv_bfloat16 *)Wq, (const __nv_bfloat16 *)kidx, scores, stride,
+                      (__nv_bfloat16 *)qidx_out);
 }
 
 }  // namespace msa

@@ -1,6 +1,8 @@
 // launch.cuh -- host-side entry points of the kernel translation units, used by abi.cu.
 #pragma once
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace msa {
@@ -16,6 +18,24 @@ struct ProfScope {
     ProfScope(const char *f, cudaStream_t s) : family(f), st(s) { prof_begin(family, st); }
     ~ProfScope() { prof_end(family, st); }
 };
+
+// Launch with programmatic stream serialization: the kernel may begin while the previous kernel
+// in the stream drains; it must call griddep_wait (ptx.cuh) as described there.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // index.cu
 cudaError_t launch_block_keys(const Prob &P, const void *K, const void *Wk, void *kidx, int64_t from_block,

@@ -139,6 +139,14 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Programmatic dependent launch.  griddep_wait blocks until the grid this one was launched after
+// has completed and its memory is visible (a no-op for a grid launched without the attribute);
+// griddep_launch lets the next grid in the stream start launching.  A kernel launched with the
+// attribute runs griddep_wait in every CTA before it reads what earlier work wrote, and before it
+// exits, so that grid completion stays ordered along the stream.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }

@@ -74,6 +74,8 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(Prob P, const float *__re
                                                        int32_t *__restrict__ out) {
     __shared__ TopkSmem<THREADS, E> S;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_wait();
+    griddep_launch();
     const int64_t rr = blockIdx.x / P.Hkv;
     const int g = blockIdx.x % P.Hkv;
     const int64_t row = P.row_begin + rr;
@@ -186,8 +188,7 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(Prob P, const float *__re
 template <int THREADS, int E>
 static cudaError_t launch_topk_t(const Prob &P, const float *scores, int64_t stride, int32_t *out, cudaStream_t st) {
     const int64_t n = (P.row_end - P.row_begin) * P.Hkv;
-    topk_kernel<THREADS, E><<<(unsigned)n, THREADS, 0, st>>>(P, scores, stride, out);
-    return cudaGetLastError();
+    return launch_pdl(topk_kernel<THREADS, E>, dim3((unsigned)n), dim3(THREADS), 0, st, P, scores, stride, out);
 }
 
 // A row has at most max_blocks - 1 candidates; rows longer than 32768 blocks are refused on the host.

@@ -212,7 +212,8 @@ msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *
  *  - Set-up: the first call on a device looks up the array's device address (with that device
  *    current) and caches it; make that first call before any CUDA stream capture.
  *  - Sharing: every call on a device uses the same array, and the array keeps the last call's
- *    contents (the call clears what must start at zero itself).  Calls that may overlap on the GPU
+ *    contents; nothing in it needs clearing between calls (its merge counters carry a per-call
+ *    generation tag).  Calls that may overlap on the GPU
  *    -- on different streams, or from different threads -- race on it: serialise them.
  *  - Every GPU that loads the library holds the 40 MiB until the process exits.
  */

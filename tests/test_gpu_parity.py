@@ -246,6 +246,23 @@ def test_decode_single_sequence():
     _decode_check(w, x)
 
 
+def test_decode_workspace_needs_no_clearing_and_repeats_bitwise():
+    # the merge counters carry a per-call generation: a workspace full of 0xFF bytes is as good as
+    # a fresh one, and the partials are combined in a fixed order, so a repeat is bit-identical
+    w = scaled_down(WORKLOADS["decode_128k"], (1, 70, 4096, 2500))
+    x = make_inputs(w, device=DEV, seed=23)
+    dc = _decode_check(w, x)
+    o1, l1 = dc.o.clone(), dc.lse.clone()
+    for _ in range(2):
+        dc.workspace.fill_(0xFF)
+        dc.o.fill_(0)
+        msa.msa_sparse_attn_decode(dc.cfg, dc.shape, x["q"], x["k"], x["v"], dc.block_idx, dc.o, dc.lse,
+                                   dc.workspace, dc.err)
+        torch.cuda.synchronize()
+        assert int(dc.err.item()) == 0
+        assert torch.equal(dc.o, o1) and torch.equal(dc.lse, l1)
+
+
 def test_decode_ragged_shape_with_ties():
     w = scaled_down(WORKLOADS["ragged_decode"], (129, 5000, 1, 3000))
     x = make_inputs(w, device=DEV, seed=9)
