@@ -183,6 +183,31 @@ def gpu_id(dist: Dist) -> str:
     return str(dist.local)
 
 
+L2_NOTE = "256 MB written, then another 256 MB read, between steps (L2 holds none of the step's data)"
+
+
+def l2_flusher():
+    """Flush L2 between timed steps: write a 256 MB buffer (2x L2), then read another one so the
+    written lines are evicted before the step starts."""
+    a = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    b = torch.zeros(32 << 20, dtype=torch.int64, device="cuda")
+
+    def flush():
+        a.fill_(1)
+        b.sum()
+    return flush
+
+
+def graph_of(fn):
+    """fn captured once in a CUDA graph (after one eager call)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
 def timed(fn, steps: int, warmup: int, dist: Dist, between=None) -> float:
     """Device milliseconds for `steps` calls of fn (CUDA events on the current stream), max over
     ranks.  `between`, if given, runs before every step outside the events (an L2 flush)."""
@@ -447,25 +472,23 @@ def secondary_measurements(args, dist, pf, x, sparse_ms, pk):
     out["dense_prefill_128k"] = {"ms": ms_dense, "tflops": dense_flops(pf.w) / (ms_dense / 1000) / 1e12,
                                  "speedup_of_sparse_step": ms_dense / sparse_ms}
     del od, ld
-    # decode at 128K: batch 32, L2 flushed between steps
+    # decode at 128K: batch 32, each step replayed from a CUDA graph, L2 flushed between steps
     wd = WORKLOADS["decode_128k"]
     xd = make_inputs(wd, device="cuda", seed=100 + dist.rank)
     dc = Decode(wd, xd)
     dc.prepare_keys()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-    between = lambda: flush.fill_(1)
-    msa.profile_reset()
-    msa.profile_enable(True)
-    ms = timed(dc.run, 20, 3, dist, between=between)
-    msa.profile_enable(False)
-    a_ms, a_n = msa.profile_read("decode_attn")
-    msa.profile_reset()
-    a_ms_launch = a_ms / max(1, a_n)
+    between = l2_flusher()
+    step = dc.graph()
+    ms = timed(step, 20, 3, dist, between=between)
+    attn = graph_of(lambda: msa.msa_sparse_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.block_idx,
+                                                       dc.o, dc.lse, dc.workspace, dc.err))
+    a_ms_launch = timed(attn.replay, 20, 3, dist, between=between) / 20
     sel_bytes = decode_selected_bytes(dc)
     gbs = sel_bytes / (a_ms_launch / 1000) / 1e9
     out["decode_128k"] = {"tokens_per_s": dist.world * wd.batch * 20 / (ms / 1000), "ms_per_step": ms / 20,
                           "attn_ms": a_ms_launch, "selected_bytes": sel_bytes, "attn_gbs": gbs,
-                          "hbm_frac": gbs / float(pk["hbm_gbs"]), "l2": "256 MB written between steps"}
+                          "hbm_frac": gbs / float(pk["hbm_gbs"]), "graph": True, "l2": L2_NOTE}
+    del attn
     ws = msa.msa_dense_attn_decode(dc.cfg, dc.shape, None, None, None, None, None, None)
     wsb = torch.empty(ws, dtype=torch.uint8, device="cuda")
     msd = timed(lambda: msa.msa_dense_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.o, dc.lse, wsb),
@@ -473,7 +496,7 @@ def secondary_measurements(args, dist, pf, x, sparse_ms, pk):
     dense_bytes = sum(wd.seqlens) * wd.Hkv * wd.D * 4
     out["dense_decode_128k"] = {"ms": msd / 5, "gbs": dense_bytes / (msd / 5 / 1000) / 1e9,
                                 "speedup_of_sparse_attn": (msd / 5) / a_ms_launch}
-    del xd, dc, flush, wsb
+    del xd, dc, wsb
     torch.cuda.empty_cache()
     return out
 
@@ -502,14 +525,14 @@ def one_million(args, dist, pk):
     xd = make_inputs(wd, device="cuda", seed=300 + dist.rank)
     dc = Decode(wd, xd)
     dc.prepare_keys()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
-    ms = timed(dc.run, 20, 3, dist, between=lambda: flush.fill_(1))
+    between = l2_flusher()
+    ms = timed(dc.graph(), 20, 3, dist, between=between)
     out["decode_1m"] = {"ms_per_step": ms / 20, "tokens_per_s": dist.world * wd.batch * 20 / (ms / 1000),
-                        "selected_bytes": decode_selected_bytes(dc)}
+                        "selected_bytes": decode_selected_bytes(dc), "graph": True, "l2": L2_NOTE}
     ws = msa.msa_dense_attn_decode(dc.cfg, dc.shape, None, None, None, None, None, None)
     wsb = torch.empty(ws, dtype=torch.uint8, device="cuda")
     msd = timed(lambda: msa.msa_dense_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.o, dc.lse, wsb),
-                3, 1, dist, between=lambda: flush.fill_(1))
+                3, 1, dist, between=between)
     out["dense_decode_1m"] = {"ms": msd / 3, "speedup_of_sparse_step": (msd / 3) / (ms / 20)}
     return out
 

@@ -101,6 +101,21 @@ class Decode:
                              self.scores, self.stride)
         self.keys_ready = True
 
+    def graph(self):
+        """Capture one decode step (index scores -> selection -> attention) in a CUDA graph and
+        return its replay function.  Every replay reads the same input tensors (refresh them in
+        place between steps) and writes the same outputs; the kernels inside are chained with
+        programmatic dependent launch."""
+        if not self.keys_ready:
+            self.prepare_keys()
+        self.run()                 # first call: per-kernel attributes set outside the capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run()
+        self._graph = g
+        return g.replay
+
     def run(self, q_idx_out=None):
         x = self.x
         if not self.keys_ready:
