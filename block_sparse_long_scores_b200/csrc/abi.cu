@@ -173,6 +173,12 @@ bool prefill_maps(const Prob &P, const void *q, const void *k, const void *v, CU
 }
 
 // Q [batch*Hq, D] -> box (64, G); cache [batch*Hkv*Lmax, D] -> box (64, B)
+// The sparse decode kernels index work items, cache rows and partial slots with 32-bit integers.
+bool decode_fits_int32(const Prob &P) {
+    const int64_t rows = (int64_t)P.batch * P.Hkv;
+    return rows < ((int64_t)1 << 26) && rows * P.k_tot < ((int64_t)1 << 31) && rows * P.Lmax < ((int64_t)1 << 31);
+}
+
 bool decode_maps(const Prob &P, const void *q, const void *k, const void *v, CUtensorMap *tq, CUtensorMap *tk,
                  CUtensorMap *tv) {
     const uint64_t dq[2] = {(uint64_t)P.D, (uint64_t)P.batch * P.Hq};
@@ -365,6 +371,7 @@ msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *
     if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
     if (shape->mode != MSA_DECODE || !workspace_bytes) return MSA_ERR_INVALID_ARG;
     const Prob P = make_prob(cfg, shape, 0, shape->batch, err_flag);
+    if (!decode_fits_int32(P)) return MSA_ERR_UNSUPPORTED;
     const size_t need = decode_stream_ws_bytes(P, num_sms());
     if (!workspace) {
         *workspace_bytes = need;
@@ -433,6 +440,7 @@ msa_status_t msa_sparse_attn_decode_noalloc(const msa_config_t *cfg, const msa_s
     if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
     if (shape->mode != MSA_DECODE) return MSA_ERR_INVALID_ARG;
     const Prob P = make_prob(cfg, shape, 0, shape->batch, err_flag);
+    if (!decode_fits_int32(P)) return MSA_ERR_UNSUPPORTED;
     if (decode_stream_ws_bytes(P, num_sms()) > kNoAllocScratchBytes) return MSA_ERR_WORKSPACE;   // beyond the fixed scratch
     if (!q || !k_cache || !v_cache || !block_idx || !o) return MSA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||

@@ -357,7 +357,8 @@ cudaError_t launch_decode(const Prob &P, const CUtensorMap &tq, const CUtensorMa
 // Streaming sparse decode.
 //
 // The selected blocks of all (sequence, kv head) rows form one work list, item
-// x = (b * Hkv + g) * k_tot + slot.  A persistent grid splits the list into contiguous ranges.  In a
+// x = (b * Hkv + g) * k_tot + slot.  A persistent grid splits the list into contiguous ranges of
+// per_cta items (all index arithmetic is 32-bit: the host refuses lists of 2^31 items or more).  In a
 // CTA a producer warp streams the range's K/V blocks through an NS-stage TMA ring and the four
 // consumer warps all read every stage: warp w takes keys [w BLK/4, (w+1) BLK/4) of the block, so the
 // chain of dependent tensor-core and softmax steps per block is a quarter of a whole block's.  Each
@@ -380,6 +381,8 @@ struct StreamSmem {
     float ob[16][D + 8];       // consumer warps' O merged at a flush (rows padded: no bank conflicts)
     float mw[kStreamConsumers][16], lw[kStreamConsumers][16];
     int lastf[32];             // tickets taken: this CTA merges the segment
+    int fslot[32][4];          // slots of the partials of segments merged on the few-partial path
+    int flist[32], nfl;        // those segments (positions in the current group of 32)
     alignas(8) uint64_t full[NS], empty[NS];
     int js[NS];
     int32_t row[256];     // sanitised block list of the producer's current (b, g)
@@ -393,28 +396,26 @@ struct StreamBufs {
     float *po;                      // [n_ctas, max_seg, 16, D] unnormalised output
     unsigned long long *tickets;    // [batch * Hkv]: (call generation << 32) | partials merged
     int max_seg;
+    int per_cta;                    // items per CTA (the last CTA may have fewer)
     uint32_t gen;                   // this call's generation (never 0)
 };
 
-// Take a segment's ticket: a count tagged with the call's generation, so that a count left by an
-// earlier call (or anything else in a fresh workspace) reads as zero and needs no clearing.
-// Returns the number of partials counted before this one.
-__device__ __forceinline__ uint32_t take_ticket(unsigned long long *t, uint32_t gen) {
+// Merge tickets are 64-bit words (call generation << 32) | partials counted.  Every CTA joins
+// the tickets of its segments when it starts: a word still tagged with another generation (left by
+// an earlier call, or anything in a fresh workspace) is reset to (gen, 0); once any CTA of this call
+// has joined, the tag matches and the word is never reset again.  A CTA adds its partial only after
+// its own join, so no count of this call is ever lost, and taking a ticket at the end is a single
+// atomic add.
+__device__ __forceinline__ void join_ticket(unsigned long long *t, uint32_t gen) {
     unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(t);
-    while (true) {
-        const uint32_t n = (uint32_t)(cur >> 32) == gen ? (uint32_t)cur : 0u;
-        const unsigned long long want = ((unsigned long long)gen << 32) | (n + 1u);
-        const unsigned long long seen = atomicCAS(t, cur, want);
-        if (seen == cur) return n;
+    while ((uint32_t)(cur >> 32) != gen) {
+        const unsigned long long seen = atomicCAS(t, cur, (unsigned long long)gen << 32);
+        if (seen == cur) break;
         cur = seen;
     }
 }
-
-__host__ __device__ __forceinline__ int64_t stream_begin(int64_t items, int64_t c, int64_t n) { return items * c / n; }
-// CTA whose range holds item x (largest c with stream_begin(c) <= x)
-__host__ __device__ __forceinline__ int64_t stream_cta_of(int64_t items, int64_t x, int64_t n) {
-    return ((x + 1) * n - 1) / items;
-}
+// Partials counted before this one.
+__device__ __forceinline__ uint32_t take_ticket(unsigned long long *t) { return (uint32_t)atomicAdd(t, 1ull); }
 
 __device__ __forceinline__ void consumers_sync() {   // the four consumer warps only
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kStreamConsumers) : "memory");
@@ -433,13 +434,13 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
     extern __shared__ unsigned char smem_raw[];
     SM &S = *reinterpret_cast<SM *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t items = (int64_t)P.batch * P.Hkv * P.k_tot;
-    const int64_t c = blockIdx.x, nc = gridDim.x;
-    const int64_t x0 = stream_begin(items, c, nc), x1 = stream_begin(items, c + 1, nc);
-    const int n = (int)(x1 - x0);
+    const int items = P.batch * P.Hkv * P.k_tot;
+    const int c = blockIdx.x, per = W.per_cta;
+    const int x0 = c * per, x1 = min(x0 + per, items);
+    const int n = x1 - x0;
     const int k_tot = P.k_tot;
-    const int64_t bg_first = x0 / k_tot;
-    const int nseg = n > 0 ? (int)((x1 - 1) / k_tot - bg_first + 1) : 0;
+    const int bg_first = x0 / k_tot, a_first = x0 - bg_first * k_tot;
+    const int nseg = n > 0 ? (x1 - 1) / k_tot - bg_first + 1 : 0;
     volatile int &fail = S.fail;
 
     if (warp == kStreamConsumers && lane == 0) {
@@ -463,16 +464,14 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
         // ------------------------------------------------------------------ producer (warp)
         // Entering a (b, g) row, the warp loads its block list once and sanitises it (out of range,
         // future or repeated -> -1, flagged); lane 0 then streams the row's blocks of this range.
-        int64_t cur_bg = -1;
-        for (int k = 0; k < n; ++k) {
-            const int64_t x = x0 + k;
-            const int64_t bg = x / k_tot;
-            const int a = (int)(x - bg * k_tot);
+        int cur_bg = -1;
+        int bg = bg_first, a = a_first;   // item x0 + k is slot a of row bg
+        for (int k = 0; k < n; ++k, a = (a + 1 == k_tot) ? 0 : a + 1, bg += (a == 0)) {
             if (bg != cur_bg) {
                 __syncwarp();
-                const int b = (int)(bg / P.Hkv);
+                const int b = bg / P.Hkv;
                 const int64_t i = ((int64_t)P.seqlens[b] - 1) / BLK;
-                const int32_t *row = block_idx + bg * k_tot;
+                const int32_t *row = block_idx + (int64_t)bg * k_tot;
                 bool canon = true;
                 int bad = 0;
                 for (int q = lane; q < k_tot; q += 32) {
@@ -511,7 +510,7 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                 if (fail) {
                 } else if (j >= 0) {
                     mbar_arrive_expect_tx(&S.full[s], 2 * DC * SM::KV_CHUNK);
-                    const int row0 = (int)(bg * P.Lmax + (int64_t)j * BLK);
+                    const int row0 = (int)((int64_t)bg * P.Lmax + (int64_t)j * BLK);
 #pragma unroll
                     for (int cc = 0; cc < DC; ++cc) {
                         tma_load_2d(S.k[s] + cc * SM::KV_CHUNK, &tm_k, &S.full[s], cc * 64, row0);
@@ -599,8 +598,12 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                     *reinterpret_cast<const float4 *>(&S.ob[e / D][e % D]);
             }
         };
-        auto load_q = [&](int64_t bg) {
-            const int b = (int)(bg / P.Hkv), g = (int)(bg % P.Hkv);
+        int loc_blk = 0, loc_lim = 0;   // the current row's local block and its last valid key
+        auto load_q = [&](int bg) {
+            const int b = bg / P.Hkv, g = bg - b * P.Hkv;
+            const int64_t pos = (int64_t)P.seqlens[b] - 1;
+            loc_blk = (int)(pos / BLK);
+            loc_lim = (int)(pos - (int64_t)loc_blk * BLK);
             const int r0 = lane >> 2, r1 = r0 + 8;
             const __nv_bfloat16 *q0 = Q + ((int64_t)b * P.Hq + (int64_t)g * P.G + r0) * D;
             const __nv_bfloat16 *q1 = Q + ((int64_t)b * P.Hq + (int64_t)g * P.G + r1) * D;
@@ -617,15 +620,15 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
         int cur = 0;
         reset();
         if (n > 0) load_q(bg_first);
-        for (int k = 0; k < n; ++k) {
+        if (warp == 1)
+            for (int sg = lane; sg < nseg; sg += 32) join_ticket(&W.tickets[bg_first + sg], W.gen);
+        int seg = 0, a = a_first;   // item x0 + k is slot a of row bg_first + seg
+        for (int k = 0; k < n; ++k, a = (a + 1 == k_tot) ? 0 : a + 1, seg += (a == 0)) {
             const int s = k % NS;
-            const int64_t x = x0 + k;
-            const int64_t bg = x / k_tot;
-            const int seg = (int)(bg - bg_first);
             if (seg != cur) {
                 flush(cur);
                 reset();
-                load_q(bg);
+                load_q(bg_first + seg);
                 cur = seg;
             }
             bool ok = fail == 0;
@@ -635,9 +638,7 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                 continue;
             }
             const int j = S.js[s];
-            const int b = (int)(bg / P.Hkv);
-            const int64_t pos = (int64_t)P.seqlens[b] - 1;
-            const int lim = (j == pos / BLK) ? (int)(pos - (int64_t)j * BLK) : BLK - 1;   // last valid key
+            const int lim = (j == loc_blk) ? loc_lim : BLK - 1;   // last valid key of the block
             if (j >= 0 && key0 <= lim) {
                 const uint32_t k_base = smem_u32(S.k[s]), v_base = smem_u32(S.v[s]);
                 float sc[NT][4];
@@ -729,6 +730,7 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
     __threadfence();
     __syncthreads();
     constexpr int kPC = 32;
+    constexpr int kFewParts = 4;
     constexpr int kThreads = 32 * (kStreamConsumers + 1);
     constexpr int kAcc = (16 * D / 4 + kThreads - 1) / kThreads;
     static_assert(2 * kPC * 16 <= 16 * (D + 8), "merge chunk must fit the flush buffer");
@@ -738,21 +740,100 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
     const int G = P.G;
     for (int s0 = 0; s0 < nseg; s0 += 32) {
         if (tid < min(32, nseg - s0)) {
-            const int64_t bg = bg_first + s0 + tid;
-            const int64_t c_first = stream_cta_of(items, bg * k_tot, nc);
-            const int64_t c_last = stream_cta_of(items, (bg + 1) * k_tot - 1, nc);
-            S.lastf[tid] = take_ticket(&W.tickets[bg], W.gen) == (uint32_t)(c_last - c_first);
+            const int bg = bg_first + s0 + tid;
+            const int c_first = bg * k_tot / per, c_last = ((bg + 1) * k_tot - 1) / per;
+            S.lastf[tid] = take_ticket(&W.tickets[bg]) == (uint32_t)(c_last - c_first);
         }
         __syncthreads();
-        for (int seg = s0; seg < min(nseg, s0 + 32); ++seg) {
+        // segments with at most kFewParts partials: their slots are listed first, then every
+        // thread loads the maxima, sums and O rows of its (segment, 4 columns) pairs in one round
+        // and combines them in registers, several segments per pass
+        const int ng = min(32, nseg - s0);
+        if (tid < ng) {
+            const int bg = bg_first + s0 + tid;
+            const int c_first = bg * k_tot / per;
+            const int np = ((bg + 1) * k_tot - 1) / per - c_first + 1;
+#pragma unroll
+            for (int p = 0; p < kFewParts; ++p) {
+                const int cc = c_first + min(p, np - 1);
+                S.fslot[tid][p] = p < np ? (cc * W.max_seg + (bg - cc * per / k_tot)) * 16 : -1;
+            }
+        }
+        if (tid == 0) {
+            int m = 0;
+            for (int t = 0; t < ng; ++t) {
+                const int bg = bg_first + s0 + t;
+                const int np = ((bg + 1) * k_tot - 1) / per - bg * k_tot / per + 1;
+                if (S.lastf[t] && np <= kFewParts) S.flist[m++] = t;
+            }
+            S.nfl = m;
+        }
+        __syncthreads();
+        if (S.nfl > 0) __threadfence();
+        const int per_seg4 = G * D / 4;
+        const int fb = max(1, (kAcc * kThreads) / per_seg4);
+        for (int f0 = 0; f0 < S.nfl; f0 += fb) {
+            const int pairs = min(fb, S.nfl - f0) * per_seg4;
+#pragma unroll
+            for (int u = 0; u < kAcc; ++u) {
+                const int q = tid + u * kThreads;
+                if (q < pairs) {
+                    const int t = S.flist[f0 + q / per_seg4], e4 = q % per_seg4;
+                    const int bg = bg_first + s0 + t;
+                    const int r = (e4 * 4) / D, col = (e4 * 4) % D;
+                    float mm[kFewParts], ll[kFewParts];
+                    float4 vv[kFewParts];
+#pragma unroll
+                    for (int p = 0; p < kFewParts; ++p) {
+                        const int sl = S.fslot[t][p];
+                        if (sl >= 0) {
+                            mm[p] = __ldcg(&W.pm[sl + r]);
+                            ll[p] = __ldcg(&W.pl[sl + r]);
+                            vv[p] = __ldcg(reinterpret_cast<const float4 *>(W.po + (int64_t)(sl + r) * D + col));
+                        } else {
+                            mm[p] = -INFINITY;
+                            ll[p] = 0.f;
+                            vv[p] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                    }
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int p = 0; p < kFewParts; ++p) M = fmaxf(M, mm[p]);
+                    float L = 0.f;
+                    float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int p = 0; p < kFewParts; ++p) {
+                        const float f = mm[p] > -INFINITY ? ex2_approx(mm[p] - M) : 0.f;
+                        L += ll[p] * f;
+                        a4.x += vv[p].x * f;
+                        a4.y += vv[p].y * f;
+                        a4.z += vv[p].z * f;
+                        a4.w += vv[p].w * f;
+                    }
+                    const float inv = L > 0.f ? 1.f / L : 0.f;
+                    const int b = bg / P.Hkv, g = bg - b * P.Hkv;
+                    const int64_t orow = (int64_t)b * P.Hq + (int64_t)g * G + r;
+                    uint2 pk;
+                    pk.x = pack_bf16(a4.x * inv, a4.y * inv);
+                    pk.y = pack_bf16(a4.z * inv, a4.w * inv);
+                    *reinterpret_cast<uint2 *>(O + orow * D + col) = pk;
+                    if (lse && col == 0)
+                        lse[orow] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+                }
+            }
+        }
+        // segments with more partials: chunked, two rounds each
+        for (int seg = s0; seg < s0 + ng; ++seg) {
             if (!S.lastf[seg - s0]) continue;   // uniform across the CTA
+            const int bg = bg_first + seg;
+            const int c_first = bg * k_tot / per;
+            const int np = ((bg + 1) * k_tot - 1) / per - c_first + 1;
+            if (np <= kFewParts) continue;      // merged above
             __threadfence();
-            const int64_t bg = bg_first + seg;
-            const int64_t c_first = stream_cta_of(items, bg * k_tot, nc);
-            const int np = (int)(stream_cta_of(items, (bg + 1) * k_tot - 1, nc) - c_first + 1);
+            const int b = bg / P.Hkv, g = bg - b * P.Hkv;
             for (int p = tid; p < np; p += kThreads) {
-                const int64_t cc = c_first + p;
-                slot_of[p] = (int)((cc * W.max_seg + (bg - stream_begin(items, cc, nc) / k_tot)) * 16);
+                const int cc = c_first + p;
+                slot_of[p] = (cc * W.max_seg + (bg - cc * per / k_tot)) * 16;
             }
             if (tid < G) {
                 S.mw[0][tid] = -INFINITY;
@@ -840,7 +921,6 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                     }
                 }
             }
-            const int b = (int)(bg / P.Hkv), g = (int)(bg % P.Hkv);
 #pragma unroll
             for (int u = 0; u < kAcc; ++u) {
                 const int e4 = tid + u * kThreads;
@@ -872,8 +952,8 @@ struct StreamCfg {
     static size_t smem() { return sizeof(StreamSmem<D, BLK, NS>) + 1024; }
 };
 
-// Grid, segment bound and workspace of the streaming decode.
-void decode_stream_geometry(const Prob &P, int num_sms, int &n_ctas, int &max_seg) {
+// Grid, items per CTA, segment bound and workspace of the streaming decode.
+void decode_stream_geometry(const Prob &P, int num_sms, int &n_ctas, int &per_cta, int &max_seg) {
     size_t smem = 0;
     if (P.D == 128 && P.B == 64) smem = StreamCfg<128, 64>::smem();
     else if (P.D == 128 && P.B == 128) smem = StreamCfg<128, 128>::smem();
@@ -882,14 +962,15 @@ void decode_stream_geometry(const Prob &P, int num_sms, int &n_ctas, int &max_se
     // the SM's 228 KB of shared memory less 1 KB reserved per resident CTA
     const int per_sm = smem + 1024 <= (size_t)114 * 1024 ? 2 : 1;
     const int64_t items = (int64_t)P.batch * P.Hkv * P.k_tot;
-    n_ctas = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms * per_sm, items));
-    const int64_t per_cta = ceil_div<int64_t>(items, n_ctas);
+    const int64_t slots = std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms * per_sm, items));
+    per_cta = (int)ceil_div<int64_t>(items, slots);
+    n_ctas = (int)std::max<int64_t>(1, ceil_div<int64_t>(items, per_cta));
     max_seg = (int)(ceil_div<int64_t>(per_cta, P.k_tot) + 1);
 }
 
 size_t decode_stream_ws_bytes(const Prob &P, int num_sms) {
-    int n_ctas, max_seg;
-    decode_stream_geometry(P, num_sms, n_ctas, max_seg);
+    int n_ctas, per_cta, max_seg;
+    decode_stream_geometry(P, num_sms, n_ctas, per_cta, max_seg);
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
     const size_t rows = (size_t)n_ctas * max_seg * 16;
     return 2 * a(sizeof(float) * rows) + a(sizeof(float) * rows * P.D) +
@@ -912,8 +993,8 @@ static cudaError_t launch_stream_t(const Prob &P, const CUtensorMap &tk, const C
 cudaError_t launch_decode_stream(const Prob &P, const CUtensorMap &tk, const CUtensorMap &tv, const void *q,
                                  const int32_t *block_idx, void *O, float *lse, void *ws, int num_sms,
                                  cudaStream_t st) {
-    int n_ctas, max_seg;
-    decode_stream_geometry(P, num_sms, n_ctas, max_seg);
+    int n_ctas, per_cta, max_seg;
+    decode_stream_geometry(P, num_sms, n_ctas, per_cta, max_seg);
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
     const size_t rows = (size_t)n_ctas * max_seg * 16;
     char *base = static_cast<char *>(ws);
@@ -924,6 +1005,7 @@ cudaError_t launch_decode_stream(const Prob &P, const CUtensorMap &tk, const CUt
     W.tickets = reinterpret_cast<unsigned long long *>(base + 2 * a(sizeof(float) * rows) +
                                                        a(sizeof(float) * rows * P.D));
     W.max_seg = max_seg;
+    W.per_cta = per_cta;
     static std::atomic<uint32_t> generation{0};
     uint32_t gen;
     do gen = ++generation; while (gen == 0);

@@ -185,7 +185,10 @@ msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t 
  * Source: as msa_sparse_attn_prefill; the digest reports decode as the second measured case.
  *  For every sequence b and query head h: the same formula with the token at position
  *  seqlens[b] - 1 and keys from k_cache/v_cache [batch, Hkv, Lmax, D];
- *  block_idx [batch, Hkv, k_tot].  Workspace: two-phase.
+ *  block_idx [batch, Hkv, k_tot].  Workspace: two-phase; its contents on entry do not matter.
+ *  Returns MSA_ERR_UNSUPPORTED (launching nothing, also on the size query) when batch x Hkv
+ *  reaches 2^26, or batch x Hkv x k_tot or batch x Hkv x Lmax reaches 2^31 (the kernel indexes
+ *  with 32-bit integers).  Repeated calls on the same inputs give bit-identical outputs.
  */
 msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *shape,
                                     const void *q, const void *k_cache, const void *v_cache,
