@@ -388,7 +388,9 @@ def main():
     achieved = flops_per_launch / (attn_launch_ms / 1000.0) / 1e12
     peak = float(pk["bf16_tflops_sustained"])
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": traffic_for("prefill_attn_128k", "block_sparse_long_scores_b200/csrc/attn_prefill.cu"),
+                # the committed figure is per launch of the default workload's 16384-row chunks
+                "traffic": (traffic_for("prefill_attn_128k", "block_sparse_long_scores_b200/csrc/attn_prefill.cu")
+                            if (w.name == "prefill_128k" and pf.chunk == 16384) else None),
                 "kernel": "sparse_prefill_attn_kernel", "launches_per_step": attn_n // args.steps,
                 "peak_kind": f"{pk_kind} bf16 sustained", "flops_per_step": flops}
     step_tflops = flops / (ms_step / 1000.0) / 1e12
