@@ -400,12 +400,14 @@ struct StreamBufs {
     uint32_t gen;                   // this call's generation (never 0)
 };
 
-// Merge tickets are 64-bit words (call generation << 32) | partials counted.  Every CTA joins
-// the tickets of its segments when it starts: a word still tagged with another generation (left by
-// an earlier call, or anything in a fresh workspace) is reset to (gen, 0); once any CTA of this call
-// has joined, the tag matches and the word is never reset again.  A CTA adds its partial only after
-// its own join, so no count of this call is ever lost, and taking a ticket at the end is a single
-// atomic add.
+// Merge tickets are 64-bit words (call generation << 32) | partials counted.  A call leaves every
+// ticket it used at 0 (the CTA that merges a segment clears its ticket).  Every CTA joins the
+// tickets of its segments when it starts: a word tagged with another generation (0 after a
+// completed call, or anything in a fresh workspace) is reset to (gen, 0); once any CTA of this call
+// has joined, the tag matches and the word is not reset again.  A CTA adds its partial only after
+// its own join, so no count of this call is lost, and taking a ticket at the end is a single atomic
+// add.  (A CUDA graph replays one generation; the clearing is what makes the next replay start
+// afresh.)
 __device__ __forceinline__ void join_ticket(unsigned long long *t, uint32_t gen) {
     unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(t);
     while ((uint32_t)(cur >> 32) != gen) {
@@ -819,6 +821,7 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                     *reinterpret_cast<uint2 *>(O + orow * D + col) = pk;
                     if (lse && col == 0)
                         lse[orow] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+                    if (e4 == 0) W.tickets[bg] = 0ull;   // merged: leave the ticket clear
                 }
             }
         }
@@ -937,6 +940,7 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                     }
                 }
             }
+            if (tid == 0) W.tickets[bg] = 0ull;   // merged: leave the ticket clear
             __syncthreads();   // shared scratch free for the next segment
         }
         __syncthreads();       // lastf free for the next group

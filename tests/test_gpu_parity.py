@@ -263,6 +263,27 @@ def test_decode_workspace_needs_no_clearing_and_repeats_bitwise():
         assert torch.equal(dc.o, o1) and torch.equal(dc.lse, l1)
 
 
+def test_decode_graph_replay_recomputes():
+    # a CUDA graph replays one set of kernel arguments: every replay must still recompute and
+    # merge (the kernel leaves its counters clear); 24 sequences make a pool of batches as well
+    lens = tuple(int(v) for v in np.random.default_rng(24).integers(2000, 6000, size=24))
+    w = scaled_down(WORKLOADS["decode_128k"], lens)
+    x = make_inputs(w, device=DEV, seed=24)
+    dc = Decode(w, x)
+    step = dc.graph()
+    g = torch.Generator(device="cpu").manual_seed(25)
+    for _ in range(3):
+        x["q"].copy_(torch.randn(x["q"].shape, generator=g).to(x["q"].dtype))
+        step()
+        torch.cuda.synchronize()
+        o_graph, lse_graph = dc.o.clone(), dc.lse.clone()
+        dc.o.fill_(0)
+        dc.run()
+        torch.cuda.synchronize()
+        assert int(dc.err.item()) == 0
+        assert torch.equal(o_graph, dc.o) and torch.equal(lse_graph, dc.lse)
+
+
 def test_decode_ragged_shape_with_ties():
     w = scaled_down(WORKLOADS["ragged_decode"], (129, 5000, 1, 3000))
     x = make_inputs(w, device=DEV, seed=9)
