@@ -90,30 +90,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
-// Non-blocking test of a phase.
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Spinning wait for short hand-offs between warps that run in step (no suspension); false if the
-// bound ran out.
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity) {
-    if (mbar_test(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_test(bar, parity)) return true;
-        if ((it & 255u) == 0 && globaltimer() - t0 > kWaitLimitNs) return false;
-    }
-}
-
 // ------------------------------------------------------------------------------ TMA and bulk
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
