@@ -9,6 +9,8 @@
 // the picks are every key > T plus the first such keys == T in ascending block order (ties go
 // to the lower block).  Ordered block-wide prefix counts then write the picks in ascending
 // block order, with the sink block in front and the local block behind them.
+#include <algorithm>
+
 #include "launch.cuh"
 
 namespace msa {
@@ -69,20 +71,49 @@ __device__ __forceinline__ int ordered_prefix(const bool (&flag)[E], int (&pos)[
     return total;
 }
 
-template <int THREADS, int E>
+// STREAM: a persistent grid walks the (row, group) problems; while it selects in one, its threads
+// copy the next problem's scores into shared memory (cp.async, double-buffered), so the load of
+// a long row (64 KB at 16384 candidates) overlaps the previous row's selection.  Otherwise one CTA
+// takes one problem and reads its scores from global memory.
+template <int THREADS, int E, bool STREAM>
 __global__ void __launch_bounds__(THREADS) topk_kernel(Prob P, const float *__restrict__ scores, int64_t stride,
                                                        int32_t *__restrict__ out) {
     __shared__ TopkSmem<THREADS, E> S;
+    extern __shared__ __align__(16) float sbuf[];   // STREAM: [2][THREADS * E]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     griddep_wait();
     griddep_launch();
-    const int64_t rr = blockIdx.x / P.Hkv;
-    const int g = blockIdx.x % P.Hkv;
+    const int64_t nprob = (P.row_end - P.row_begin) * P.Hkv;
+    const int64_t step = STREAM ? (int64_t)gridDim.x : nprob;
+    // scores of problem t: candidates j < i of its row; copied whole 16-byte chunks from j = 0
+    auto prefetch = [&](int64_t t, int b) {
+        const int64_t rr = t / P.Hkv;
+        const int gg = (int)(t % P.Hkv);
+        const int64_t ii = row_geo(P, P.row_begin + rr).pos / P.B;
+        const float *src = scores + (rr * P.Hkv + gg) * stride;
+        float *dst = sbuf + (size_t)b * THREADS * E;
+        for (int64_t q = tid; q < (ii + 3) / 4; q += THREADS) cp_async_16(dst + 4 * q, src + 4 * q);
+        cp_async_commit();
+    };
+    if (STREAM && blockIdx.x < nprob) prefetch(blockIdx.x, 0);
+    int it = 0;
+    for (int64_t t = blockIdx.x; t < nprob; t += step, ++it) {
+    if (STREAM) {
+        if (t + step < nprob) {
+            prefetch(t + step, (it + 1) & 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+    }
+    const int64_t rr = t / P.Hkv;
+    const int g = (int)(t % P.Hkv);
     const int64_t row = P.row_begin + rr;
     const RowGeo geo = row_geo(P, row);
     const int64_t i = geo.pos / P.B;
     const int s = P.use_sink;
-    const float *Sr = scores + (rr * P.Hkv + g) * stride;
+    const float *Sr = STREAM ? sbuf + (size_t)(it & 1) * THREADS * E : scores + (rr * P.Hkv + g) * stride;
     int32_t *o = out + (rr * P.Hkv + g) * (int64_t)P.k_tot;
 
     // key 0 marks "no candidate" (past the range, or a NaN score); every number maps above 0
@@ -183,12 +214,32 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(Prob P, const float *__re
         o[sinkoff + n_sel] = (int32_t)i;
     }
     for (int q = sinkoff + n_sel + 1 + tid; q < P.k_tot; q += THREADS) o[q] = -1;
+    if (STREAM) __syncthreads();   // this buffer is refilled two problems later
+    }
 }
 
 template <int THREADS, int E>
 static cudaError_t launch_topk_t(const Prob &P, const float *scores, int64_t stride, int32_t *out, cudaStream_t st) {
     const int64_t n = (P.row_end - P.row_begin) * P.Hkv;
-    return launch_pdl(topk_kernel<THREADS, E>, dim3((unsigned)n), dim3(THREADS), 0, st, P, scores, stride, out);
+    return launch_pdl(topk_kernel<THREADS, E, false>, dim3((unsigned)n), dim3(THREADS), 0, st, P, scores, stride,
+                      out);
+}
+
+// Long rows: one persistent CTA per SM, scores prefetched into shared memory.
+template <int THREADS, int E>
+static cudaError_t launch_topk_stream_t(const Prob &P, const float *scores, int64_t stride, int32_t *out,
+                                        cudaStream_t st) {
+    const int64_t n = (P.row_end - P.row_begin) * P.Hkv;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const size_t smem = 2 * sizeof(float) * THREADS * E;
+    auto kern = topk_kernel<THREADS, E, true>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return e;
+    const unsigned grid = (unsigned)std::min<int64_t>(n, sms);
+    return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, st, P, scores, stride, out);
 }
 
 // A row has at most max_blocks - 1 candidates; rows longer than 32768 blocks are refused on the host.
@@ -199,7 +250,7 @@ cudaError_t launch_select_topk(const Prob &P, const float *scores, int64_t strid
     if (nmax <= 128 * 4) return launch_topk_t<128, 4>(P, scores, stride, out, st);
     if (nmax <= 128 * 16) return launch_topk_t<128, 16>(P, scores, stride, out, st);
     if (nmax <= 256 * 32) return launch_topk_t<256, 32>(P, scores, stride, out, st);
-    if (nmax <= 512 * 32) return launch_topk_t<512, 32>(P, scores, stride, out, st);
+    if (nmax <= 512 * 32) return launch_topk_stream_t<512, 32>(P, scores, stride, out, st);
     if (nmax <= 1024 * 32) return launch_topk_t<1024, 32>(P, scores, stride, out, st);
     return cudaErrorInvalidValue;
 }
