@@ -7,14 +7,16 @@
 // 64, so the contraction uses warp-level mma.sync (m16n8k16, bf16 in, fp32 accumulate) on
 // 128-byte-swizzled tiles that TMA streams in; the tensor pipe is never this kernel's limit.
 //
-// Grid (ctas_per_bg, Hkv, batch).  A CTA has NW warps; in each round every warp takes one block
-// (TMA into its own K/V slot), computes S = Q K^T, an online-softmax update and O += P V.  The
-// warps' states are merged in shared memory into one split partial (m, l, O) per CTA.  The last
-// CTA of a (sequence, kv head) to finish (atomic ticket, no waiting) merges all splits:
+// Two kernels.  decode_attn_kernel (below; used for the dense decode baseline): grid
+// (ctas_per_bg, Hkv, batch), a CTA has NW warps, in each round every warp takes one block (TMA into
+// its own K/V slot), computes S = Q K^T, an online-softmax update and O += P V; the warps' states
+// are merged in shared memory into one split partial (m, l, O) per CTA, and the last CTA of a
+// (sequence, kv head) to finish (atomic ticket, no waiting) merges all splits:
 //   m = max_c m_c;  l = sum_c l_c 2^(m_c - m);  O = sum_c O_c 2^(m_c - m) / l;  lse = (m + log2 l) ln 2
-// (scores are kept in log2 units: t = scale * log2(e) * q.k).
+// (scores are kept in log2 units: t = scale * log2(e) * q.k).  decode_stream_kernel (further down;
+// the sparse decode) streams the whole batch's selected blocks through a persistent grid and
+// merges with the same rule.
 #include <algorithm>
-
 #include <atomic>
 
 #include "launch.cuh"
