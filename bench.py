@@ -52,6 +52,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--with-1m", action="store_true", help="also time the 1M-token workloads")
+    ap.add_argument("--with-ragged", action="store_true", help="also time the ragged prefill and decode workloads")
     ap.add_argument("--seq-len", type=int, default=0, help="scaled-down sequence (profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -407,6 +408,8 @@ def main():
         secondary = secondary_measurements(args, dist, pf, x, ms_step, pk)
         if args.with_1m:
             secondary.update(one_million(args, dist, pk))
+        if args.with_ragged:
+            secondary.update(ragged(args, dist, pk))
 
     # --- CPU oracle baseline (rank 0, N=1 only)
     cpu_baseline = None
@@ -536,6 +539,42 @@ def one_million(args, dist, pk):
     msd = timed(lambda: msa.msa_dense_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.o, dc.lse, wsb),
                 3, 1, dist, between=between)
     out["dense_decode_1m"] = {"ms": msd / 3, "speedup_of_sparse_step": (msd / 3) / (ms / 20)}
+    return out
+
+
+def ragged(args, dist, pk):
+    """The ragged workloads: 16 sequences of 1K-256K tokens, 64 q / 8 kv heads, D 64, block 128,
+    top-k 32 + local, index keys from 8 discrete vectors (exact score ties)."""
+    from block_sparse_long_scores_b200 import msa
+    from block_sparse_long_scores_b200.pipeline import Decode, Prefill
+    from block_sparse_long_scores_b200.workloads import WORKLOADS, make_inputs
+
+    out = {}
+    w = WORKLOADS["ragged_prefill"]
+    x = make_inputs(w, device="cuda", seed=400 + dist.rank)
+    pf = Prefill(w, x, chunk_rows=args.chunk_rows)
+    ms = timed(pf.run, 1, 1, dist)
+    flops = selected_flops(pf)
+    out["ragged_prefill"] = {"ms": ms, "tokens": pf.shape.total_rows,
+                             "tokens_per_s": dist.world * pf.shape.total_rows / (ms / 1000),
+                             "tflops_selected": flops / (ms / 1000) / 1e12}
+    del x, pf
+    torch.cuda.empty_cache()
+    wd = WORKLOADS["ragged_decode"]
+    xd = make_inputs(wd, device="cuda", seed=500 + dist.rank)
+    dc = Decode(wd, xd)   # its block keys are the workload's discrete ones (given, not recomputed)
+    between = l2_flusher()
+    ms = timed(dc.graph(), 20, 3, dist, between=between)
+    attn = graph_of(lambda: msa.msa_sparse_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.block_idx,
+                                                       dc.o, dc.lse, dc.workspace, dc.err))
+    a_ms = timed(attn.replay, 20, 3, dist, between=between) / 20
+    sel = decode_selected_bytes(dc)
+    out["ragged_decode"] = {"ms_per_step": ms / 20, "tokens_per_s": dist.world * wd.batch * 20 / (ms / 1000),
+                            "attn_ms": a_ms, "selected_bytes": sel, "attn_gbs": sel / (a_ms / 1000) / 1e9,
+                            "hbm_frac": sel / (a_ms / 1000) / 1e9 / float(pk["hbm_gbs"]), "graph": True,
+                            "l2": L2_NOTE}
+    del attn, xd, dc
+    torch.cuda.empty_cache()
     return out
 
 
