@@ -167,7 +167,8 @@ __global__ void prefill_tiles_kernel(int64_t L, int tpt, const int32_t *__restri
 //   warps 2-3   query gather: cp.async of each token's G head rows into the swizzled operand
 //   warp 1      MMA issuer: S = Q K^T into one of 2 TMEM S buffers, O = P V into one of 2 TMEM O
 //               buffers; MMA1 of tile t+1 is issued before MMA2 of tile t
-//   warps 4-7   softmax: S (TMEM) -> row max/sum -> bf16 P tile in shared memory, one thread per row
+//   warps 4-7   softmax: S (TMEM) -> row max/sum -> bf16 P tile in TMEM, one thread per row (P never
+//               touches shared memory: the kernel's shared-memory traffic is close to its bandwidth)
 //   warps 8-11  epilogue: O (TMEM) -> unnormalised bf16 partial + (max, sum) -> global through
 //               per-warp shared-memory staging
 // Hand-offs are mbarriers; "empty" barriers start free (first wait on parity 1 passes).
@@ -183,15 +184,15 @@ struct AttnShape {
     static constexpr int KV_CHUNK = BLK * 128;    // BLK rows x 128 B
     static constexpr int KV_STAGE = DC * KV_CHUNK;
     static constexpr int P_STAGE = BC * Q_CHUNK;
-    // Query gathers arrive ~2 us after issue, so the ring keeps several in flight; K/V change only
-    // every few dozen tiles, so one K/V stage is enough where shared memory is short.
+    // Query gathers arrive ~2 us after issue, so the ring keeps several in flight; two K/V stages
+    // let the next list's block load while the current list's tiles run.
     static constexpr int NQ = 4;
-    static constexpr int NKV = (D == 128) ? 1 : 2;
+    static constexpr int NKV = 2;
     static constexpr int NCTX = 8;
-    // TMEM columns: S 2 x BLK, O 2 x D (fp32)
-    static constexpr int TMEM_S0 = 0, TMEM_O0 = 2 * BLK;
+    // TMEM columns: S 2 x BLK and O 2 x D (fp32), P 2 x BLK/2 (bf16 pairs: the A operand of O = P V)
+    static constexpr int TMEM_S0 = 0, TMEM_O0 = 2 * BLK, TMEM_P0 = 2 * BLK + 2 * D;
     static constexpr int TMEM_COLS = 512;
-    static_assert(2 * BLK + 2 * D <= TMEM_COLS, "TMEM budget");
+    static_assert(TMEM_P0 + BLK <= TMEM_COLS, "TMEM budget");
 };
 
 constexpr int kSeqCache = 256;   // sequences whose offsets the attention kernel keeps in smem
@@ -208,7 +209,6 @@ struct AttnSmem {
     using A = AttnShape<D, BLK, G>;
     alignas(1024) unsigned char q[A::NQ][A::Q_STAGE];
     alignas(1024) unsigned char kv[A::NKV][2][A::KV_STAGE];
-    alignas(1024) unsigned char p[2][A::P_STAGE];
     TileCtx ctx[A::NCTX];
     float2 ml[4][128];                     // softmax -> epilogue, ring of 4 (see ml_full)
     int32_t cu_blocks[kSeqCache + 1], cu_seqlens[kSeqCache + 1];   // small batches: sequence table
@@ -436,13 +436,14 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
                 if (!wait_or_fail(&S.p_full[ps], (i >> 1) & 1, &S.fail)) return false;
                 if (!wait_or_fail(&S.o_empty[ps], ((i >> 1) & 1) ^ 1, &S.fail)) return false;
                 tc_fence_after();
-                const uint32_t p0 = smem_u32(S.p[ps]), v0 = smem_u32(S.kv[pend_kvs][1]);
+                const uint32_t v0 = smem_u32(S.kv[pend_kvs][1]);
+                const uint32_t p_tmem = tmem + A::TMEM_P0 + ps * (BLK / 2);
 #pragma unroll
                 for (int kc = 0; kc < A::BC; ++kc)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + A::TMEM_O0 + ps * D, sdesc(p0 + kc * A::Q_CHUNK + kk * 32, 16, 1024),
-                                  sdesc(v0 + (kc * 64 + kk * 16) * 128, A::KV_CHUNK, 1024), idesc_o, (kc | kk) != 0);
+                    for (int kk = 0; kk < 4; ++kk)   // A = P from TMEM: 8 columns hold 16 keys
+                        umma_bf16_ts(tmem + A::TMEM_O0 + ps * D, p_tmem + (kc * 4 + kk) * 8,
+                                     sdesc(v0 + (kc * 64 + kk * 16) * 128, A::KV_CHUNK, 1024), idesc_o, (kc | kk) != 0);
                 umma_commit(&S.o_full[ps]);
                 umma_commit(&S.p_empty[ps]);
                 if (pend_last) umma_commit(&S.kv_empty[pend_kvs]);
@@ -547,19 +548,14 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
                 }
 #pragma unroll
                 for (int x = 0; x < 32; ++x) l += pv[x];
-                unsigned char *pc = S.p[ts] + (cc >> 1) * A::Q_CHUNK;
+                uint32_t pk[16];   // 32 keys of the P row as bf16 pairs (keys 2c, 2c+1 in column c)
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 w;
-                    w.x = pack_bf16(pv[8 * q + 0], pv[8 * q + 1]);
-                    w.y = pack_bf16(pv[8 * q + 2], pv[8 * q + 3]);
-                    w.z = pack_bf16(pv[8 * q + 4], pv[8 * q + 5]);
-                    w.w = pack_bf16(pv[8 * q + 6], pv[8 * q + 7]);
-                    *reinterpret_cast<uint4 *>(pc + sw128(row, (cc & 1) * 4 + q)) = w;
-                }
+                for (int x = 0; x < 16; ++x) pk[x] = pack_bf16(pv[2 * x], pv[2 * x + 1]);
+                tmem_st16(tmem + lane_base + A::TMEM_P0 + ts * (BLK / 2) + cc * 16, pk);
             }
+            tmem_st_wait();
             S.ml[i & 3][row] = make_float2(m2, l);
-            fence_async_smem();   // P is read by the tensor core (async proxy)
+            tc_fence_before();   // P is read by the tensor core after the hand-off
             mbar_arrive(&S.p_full[ts]);
             mbar_arrive(&S.ml_full[i & 3]);
         }
