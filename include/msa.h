@@ -188,7 +188,9 @@ msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t 
  *  block_idx [batch, Hkv, k_tot].  Workspace: two-phase; its contents on entry do not matter.
  *  Returns MSA_ERR_UNSUPPORTED (launching nothing, also on the size query) when batch x Hkv
  *  reaches 2^26, or batch x Hkv x k_tot or batch x Hkv x Lmax reaches 2^31 (the kernel indexes
- *  with 32-bit integers).  Repeated calls on the same inputs give bit-identical outputs.
+ *  with 32-bit integers).  Repeated calls on the same inputs give bit-identical outputs, and the
+ *  call may be captured in a CUDA graph: every replay recomputes and merges (its merge counters
+ *  are left clear after each call).
  */
 msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *shape,
                                     const void *q, const void *k_cache, const void *v_cache,
