@@ -79,15 +79,16 @@ bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, 
 }
 
 int num_sms() {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64];   // zero-initialised (static storage); 0 = not looked up yet
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!cache[dev]) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (!n) {
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cache[dev] = n > 0 ? n : 148;
+        n = n > 0 ? n : 148;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 // --------------------------------------------------------------------------- validation
