@@ -128,3 +128,54 @@ def test_index_scores_rejects_bad_stride(L):
         rc = L.msa_index_scores(ctypes.byref(cfg), ctypes.byref(shape), fake, fake, fake, fake, fake, 0, 0, 10, fake,
                                 stride, None, None)
         assert rc == 1
+
+
+def _decode_shape(batch, Lmax, B=64):
+    return msa.Shape(msa.MSA_DECODE, batch, None, None, 0x10000, batch, 0, Lmax, (Lmax + B - 1) // B)
+
+
+def _decode_ws(L, cfg, shape):
+    n = ctypes.c_size_t(0)
+    rc = L.msa_sparse_attn_decode(ctypes.byref(cfg), ctypes.byref(shape), None, None, None, None, None, None, None,
+                                  ctypes.byref(n), None, None)
+    return rc, n.value
+
+
+def test_decode_workspace_follows_the_split_geometry(L):
+    # Without a GPU the library sizes for 148 SMs; (head_dim 128, 64-token blocks) runs 2 CTAs per
+    # SM.  Items = batch x Hkv x k_tot split into equal runs; one (m, l, O) partial slot of 16 rows
+    # per CTA and segment it touches; one 64-bit merge counter per (sequence, kv head).
+    def expected(batch, Hkv, k_tot, D):
+        items = batch * Hkv * k_tot
+        slots = min(148 * 2, items)
+        per = -(-items // slots)
+        n_ctas = -(-items // per)
+        max_seg = -(-per // k_tot) + 1
+        rows = n_ctas * max_seg * 16
+        a = lambda x: (x + 255) & ~255
+        return 2 * a(4 * rows) + a(4 * rows * D) + a(8 * batch * Hkv)
+
+    rc, n = _decode_ws(L, _cfg(), _decode_shape(32, 131072))                    # decode 128K
+    assert rc == 0 and n == expected(32, 4, 66, 128)
+    assert 4.5 * 2**20 < n < 4.9 * 2**20                                        # "4.7 MiB" in the header
+    rc, n = _decode_ws(L, _cfg(n_topk=128), _decode_shape(8, 1 << 20))         # decode 1M
+    assert rc == 0 and n == expected(8, 4, 130, 128)
+
+
+def test_noalloc_decode_refuses_problems_beyond_its_scratch_on_the_host(L):
+    cfg = _cfg()
+    args = [None] * 6 + [None, None]   # q, k, v, block_idx, o, lse, err_flag, stream
+    # 4096 sequences x 4 kv heads x 66 slots: ~140 MiB of partials > the 40 MiB array
+    rc = L.msa_sparse_attn_decode_noalloc(ctypes.byref(cfg), ctypes.byref(_decode_shape(4096, 64)), *args)
+    assert rc == 3
+    # the 128K decode workload fits: it passes the size check and stops at the null pointers
+    rc = L.msa_sparse_attn_decode_noalloc(ctypes.byref(cfg), ctypes.byref(_decode_shape(32, 131072)), *args)
+    assert rc == 1
+
+
+def test_decode_refuses_problems_beyond_32_bit_indexing(L):
+    # batch x Hkv x Lmax = 8192 x 4 x 65536 = 2^31 cache rows: refused on the size query as well
+    rc, _ = _decode_ws(L, _cfg(), _decode_shape(8192, 65536))
+    assert rc == 2
+    rc, _ = _decode_ws(L, _cfg(), _decode_shape(4096, 65536))                  # 2^30 rows: accepted
+    assert rc == 0
