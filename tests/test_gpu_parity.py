@@ -374,14 +374,16 @@ def _prefill_sampled_check(w, x, rows, chunk_rows):
 def test_prefill_1m_full_size_sampled():
     w = WORKLOADS["prefill_1m"]
     x = make_inputs(w, device=DEV)
-    _prefill_sampled_check(w, x, sample_rows(w, 192, seed=1), chunk_rows=16384)
+    # 4096 sampled rows, including the first and last 64 of the sequence
+    _prefill_sampled_check(w, x, sample_rows(w, 4096, seed=1), chunk_rows=16384)
 
 
 @pytest.mark.slow
 def test_ragged_prefill_full_size_sampled():
     w = WORKLOADS["ragged_prefill"]
     x = make_inputs(w, device=DEV)
-    _prefill_sampled_check(w, x, sample_rows(w, 1024, seed=2), chunk_rows=16384)
+    # 4096 sampled rows, including the first and last 64 of every sequence
+    _prefill_sampled_check(w, x, sample_rows(w, 4096, seed=2), chunk_rows=16384)
 
 
 def _decode_sampled_check(w, x):
