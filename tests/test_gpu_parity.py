@@ -284,6 +284,38 @@ def test_decode_graph_replay_recomputes():
         assert torch.equal(o_graph, dc.o) and torch.equal(lse_graph, dc.lse)
 
 
+def test_decode_bad_and_unordered_block_ids_are_flagged_and_skipped():
+    # the decode kernel sanitises each block list once per CTA: out-of-range ids and repeats are
+    # skipped and flagged, any order is accepted (the selection is a set)
+    w = scaled_down(WORKLOADS["decode_128k"], (300, 5000, 4096, 2))
+    x = make_inputs(w, device=DEV, seed=26)
+    dc = Decode(w, x)
+    dc.run()
+    torch.cuda.synchronize()
+    assert int(dc.err.item()) == 0
+    sel = dc.block_idx.cpu().numpy()
+    bad, clean = sel.copy(), sel.copy()
+    bad[1, 0] = sel[1, 0][::-1]                        # valid, descending, padding first
+    v = np.flatnonzero(sel[1, 1] >= 0)
+    bad[1, 1, v[-1]] = sel[1, 1, v[0]]                  # a repeat of the first block replaces the last
+    clean[1, 1, v[-1]] = -1
+    v = np.flatnonzero(sel[2, 2] >= 0)
+    bad[2, 2, v[1]] = 99999                            # beyond the local block
+    clean[2, 2, v[1]] = -1
+    bad[0, 3, 1] = -7                                   # negative other than -1
+    clean[0, 3, 1] = -1
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, lse = torch.empty_like(dc.o), torch.empty_like(dc.lse)
+    msa.msa_sparse_attn_decode(dc.cfg, dc.shape, x["q"], x["k"], x["v"], torch.as_tensor(bad, device=DEV), o, lse,
+                               dc.workspace, err)
+    torch.cuda.synchronize()
+    flags = int(err.item())
+    assert flags & 1 and flags & 2, flags
+    xc = cpu(x)
+    O_ref, L_ref = orc.sparse_attn(oracle_shape(w, xc), xc["q"], xc["k"], xc["v"], clean, np.arange(w.batch))
+    check_attention(o.float().cpu().numpy(), O_ref, lse.cpu().numpy(), L_ref)
+
+
 def test_decode_ragged_shape_with_ties():
     w = scaled_down(WORKLOADS["ragged_decode"], (129, 5000, 1, 3000))
     x = make_inputs(w, device=DEV, seed=9)
