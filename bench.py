@@ -451,10 +451,12 @@ def emit(args, dist, w, T, pf, value, ms_step, roofline, cpu_baseline, e2e, laun
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{w.name}: 1 x {T} tokens, {w.Hq} q / {w.Hkv} kv heads, D {w.D}, "
-                                   f"block {w.B}, top-k {w.n_topk} + sink + local, index dim {w.d}",
+            "config": {"workload": f"{w.name}: {len(w.seqlens)} x {T // len(w.seqlens)} tokens"
+                                   f"{' (ragged)' if len(set(w.seqlens)) > 1 else ''}, {w.Hq} q / {w.Hkv} kv "
+                                   f"heads, D {w.D}, block {w.B}, top-k {w.n_topk}"
+                                   f"{' + sink' if w.use_sink else ''} + local, index dim {w.d}",
                        "global_batch": dist.world, "seq_len": T, "chunk_rows": pf.chunk,
-                       "l2": "inputs exceed L2 (Q 1.07 GB read per step); no flush",
+                       "l2": f"inputs exceed L2 (Q {T * w.Hq * w.D * 2 / 1e9:.2f} GB read per step); no flush",
                        "parallelism": f"dp{dist.world} (one independent sequence per rank)"},
             "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk, "step_tflops_selected": step_tflops, "kernel_ms_per_step": fam,

@@ -50,3 +50,36 @@ def test_two_rank_max_and_weak_scaling_rate():
 def test_single_process_rate():
     import bench
     assert bench.throughput(1, 131072, 5, 250.0) == pytest.approx(131072 * 5 / 0.25)
+
+
+def test_emitted_line_carries_the_contract_keys(capsys):
+    # the JSON line the driver parses: every key and its type, built from fake measurements
+    import json
+    from types import SimpleNamespace
+    import bench
+    from block_sparse_long_scores_b200.workloads import WORKLOADS
+
+    w = WORKLOADS["prefill_128k"]
+    roofline = {"bound": "tensor", "achieved": 400.0, "peak": 1414.8, "unit": "TFLOP/s", "frac": 400.0 / 1414.8,
+                "traffic": 9.9e9}
+    cpu = {"value": 300.0, "unit": "tokens/s", "cores": 16, "kind": "oracle", "sample": "rows"}
+    e2e = {"value": 1.5e6, "unit": "tokens/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 1}
+    clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    bench.emit(SimpleNamespace(steps=5, warmup=3), SimpleNamespace(rank=0, world=1), w, 131072,
+               SimpleNamespace(chunk=16384), 3.1e6, 41.5, roofline, cpu, e2e, 325, clk, 213.0, {}, {})
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key, typ in [("metric", str), ("value", float), ("unit", str), ("n_gpus", int), ("steps", int),
+                     ("warmup", int), ("ms_per_step", float), ("higher_is_better", bool), ("scaling", str),
+                     ("dtype", str), ("data", str), ("config", dict), ("roofline", dict), ("cpu_baseline", dict),
+                     ("e2e", dict), ("gpu_launches", int), ("clocks", dict)]:
+        assert isinstance(line[key], typ), key
+    assert "vs_baseline" in line and line["scaling"] == "weak" and line["higher_is_better"] is True
+    assert set(roofline) <= set(line["roofline"]) and line["cpu_baseline"]["kind"] == "oracle"
+    assert {"workload", "global_batch", "seq_len", "l2"} <= set(line["config"])
+    assert "1.07 GB" in line["config"]["l2"] and "+ sink" in line["config"]["workload"]
+    # the ragged workload has no sink and unequal lengths
+    wr = WORKLOADS["ragged_prefill"]
+    bench.emit(SimpleNamespace(steps=1, warmup=1), SimpleNamespace(rank=0, world=1), wr, sum(wr.seqlens),
+               SimpleNamespace(chunk=16384), 1.0, 1.0, roofline, None, None, 1, clk, 1.0, {}, {})
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert "+ sink" not in line["config"]["workload"] and "(ragged)" in line["config"]["workload"]
