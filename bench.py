@@ -335,7 +335,7 @@ def reference_arm(args, dist: Dist):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall * 1000 / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "seq_len": w.total_rows},
+            "config": workload_config(w, w.total_rows, min(args.chunk_rows, w.total_rows), dist.world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -444,6 +444,17 @@ def end_to_end(args, dist, pf, x, T):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / args.steps}
 
 
+def workload_config(w, T: int, chunk: int, world: int) -> dict:
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": f"{w.name}: {len(w.seqlens)} x {T // len(w.seqlens)} tokens"
+                        f"{' (ragged)' if len(set(w.seqlens)) > 1 else ''}, {w.Hq} q / {w.Hkv} kv heads, "
+                        f"D {w.D}, block {w.B}, top-k {w.n_topk}{' + sink' if w.use_sink else ''} + local, "
+                        f"index dim {w.d}",
+            "global_batch": world, "seq_len": T, "chunk_rows": chunk,
+            "l2": f"inputs exceed L2 (Q {T * w.Hq * w.D * 2 / 1e9:.2f} GB read per step); no flush",
+            "parallelism": f"dp{world} (one independent sequence per rank)"}
+
+
 def emit(args, dist, w, T, pf, value, ms_step, roofline, cpu_baseline, e2e, launches, clk, step_tflops, fam,
          secondary):
     if dist.rank != 0:
@@ -451,13 +462,7 @@ def emit(args, dist, w, T, pf, value, ms_step, roofline, cpu_baseline, e2e, laun
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{w.name}: {len(w.seqlens)} x {T // len(w.seqlens)} tokens"
-                                   f"{' (ragged)' if len(set(w.seqlens)) > 1 else ''}, {w.Hq} q / {w.Hkv} kv "
-                                   f"heads, D {w.D}, block {w.B}, top-k {w.n_topk}"
-                                   f"{' + sink' if w.use_sink else ''} + local, index dim {w.d}",
-                       "global_batch": dist.world, "seq_len": T, "chunk_rows": pf.chunk,
-                       "l2": f"inputs exceed L2 (Q {T * w.Hq * w.D * 2 / 1e9:.2f} GB read per step); no flush",
-                       "parallelism": f"dp{dist.world} (one independent sequence per rank)"},
+            "config": workload_config(w, T, pf.chunk, dist.world),
             "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk, "step_tflops_selected": step_tflops, "kernel_ms_per_step": fam,
             "secondary": secondary}

@@ -83,3 +83,12 @@ def test_emitted_line_carries_the_contract_keys(capsys):
                SimpleNamespace(chunk=16384), 1.0, 1.0, roofline, None, None, 1, clk, 1.0, {}, {})
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert "+ sink" not in line["config"]["workload"] and "(ragged)" in line["config"]["workload"]
+
+
+def test_both_arms_describe_the_same_config():
+    import bench
+    from block_sparse_long_scores_b200.workloads import WORKLOADS
+    w = WORKLOADS["prefill_128k"]
+    ours = bench.workload_config(w, 131072, 16384, 1)
+    ref = bench.workload_config(w, w.total_rows, min(16384, w.total_rows), 1)
+    assert ours == ref
