@@ -14,8 +14,12 @@ Besides the headline line items, the line carries:
   roofline      the dominant kernel (sparse prefill attention, tensor-bound): selected-block FLOPs
                 per launch / its launch time from CUDA events recorded around it in the timed region
   cpu_baseline  the fp64 CPU oracle on a bounded sample of rows of the same workload (rank 0, N=1)
-  e2e           the same step with host->device copies of Q/K/V/W and device->host of O/lse
-  secondary     decode at 128K (HBM roofline on selected-block bytes) and the dense GQA baselines
+  e2e           the same step from pinned host buffers to pinned host buffers (Q/K/V/W in, O/lse
+                out), chunk copies overlapping other chunks' compute
+  secondary     decode at 128K and 1M (whole step, and the attention kernel against the HBM roofline
+                on selected-block bytes), prefill at 1M, the ragged prefill and decode workloads, and
+                the dense causal GQA baselines at 128K and 1M with the sparse path's speed-up over
+                them; with its own clock record (--quick skips the 1M and ragged workloads)
 """
 from __future__ import annotations
 
@@ -51,8 +55,7 @@ def parse_args():
     ap.add_argument("--chunk-rows", type=int, default=16384)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
     ap.add_argument("--no-secondary", action="store_true")
-    ap.add_argument("--with-1m", action="store_true", help="also time the 1M-token workloads")
-    ap.add_argument("--with-ragged", action="store_true", help="also time the ragged prefill and decode workloads")
+    ap.add_argument("--quick", action="store_true", help="skip the 1M-token and ragged workloads")
     ap.add_argument("--seq-len", type=int, default=0, help="scaled-down sequence (profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -364,23 +367,23 @@ def main():
     T = pf.shape.total_rows
     clocks = ClockSampler(gpu_id(dist))
 
-    # --- headline: inputs resident in HBM
+    # --- headline: inputs resident in HBM.  Inside the timed region only the dominant kernel is
+    # bracketed by CUDA events (for the roofline); the per-family split comes from a separate pass.
+    clocks.start()
     for _ in range(args.warmup):
         pf.run()
     torch.cuda.synchronize()
-    clocks.start()
     msa.profile_reset()
+    msa.profile_only("prefill_attn")
     msa.profile_enable(True)
     n0 = msa.launch_count()
     ms = timed(pf.run, args.steps, 0, dist)
     launches = msa.launch_count() - n0
     msa.profile_enable(False)
+    msa.profile_only(None)
     attn_ms, attn_n = msa.profile_read("prefill_attn")
-    fam = {}
-    for f in ("block_keys", "index_scores", "select_topk", "prefill_lists", "prefill_attn", "prefill_combine"):
-        t, n = msa.profile_read(f)
-        fam[f] = round(t / args.steps, 3)
     msa.profile_reset()
+    fam = family_split(msa, pf)
     flops = selected_flops(pf)
     ms_step = ms / args.steps
     value = throughput(dist.world, T, args.steps, ms)
@@ -402,15 +405,7 @@ def main():
         e2e = end_to_end(args, dist, pf, x, T)
     clk = clocks.stop()
 
-    # --- secondary: decode 128K and the dense baselines (rank 0 reports, every rank runs)
-    secondary = {}
-    if not args.no_secondary:
-        secondary = secondary_measurements(args, dist, pf, x, ms_step, pk)
-        if args.with_1m:
-            secondary.update(one_million(args, dist, pk))
-        if args.with_ragged:
-            secondary.update(ragged(args, dist, pk))
-
+    chunk = pf.chunk
     # --- CPU oracle baseline (rank 0, N=1 only)
     cpu_baseline = None
     if dist.world == 1 and args.cpu_seconds > 0:
@@ -420,12 +415,48 @@ def main():
                         "sample": f"{n} random rows of {w.name} (whole path per row: index query, scores, "
                                   f"top-k, attention) plus block keys of all {pf.shape.total_blocks} blocks "
                                   f"amortised per row, fp64, ~{args.cpu_seconds:.0f} s"}
-    emit(args, dist, w, T, pf, value, ms_step, roofline, cpu_baseline, e2e, launches, clk, step_tflops, fam,
+        del xc
+
+    # --- secondary: decode 128K, 1M, ragged and the dense baselines (rank 0 reports, every rank
+    # runs), with their own clock record
+    secondary = {}
+    if not args.no_secondary:
+        sec_clocks = ClockSampler(gpu_id(dist))
+        sec_clocks.start()
+        secondary = secondary_measurements(args, dist, pf, x, ms_step, pk)
+        del pf, x
+        torch.cuda.empty_cache()
+        if not args.quick:
+            secondary.update(one_million(args, dist, pk))
+            secondary.update(ragged(args, dist, pk))
+        secondary["clocks"] = sec_clocks.stop()
+
+    emit(args, dist, w, T, chunk, value, ms_step, roofline, cpu_baseline, e2e, launches, clk, step_tflops, fam,
          secondary)
     dist.close()
 
 
+def family_split(msa, pf) -> dict:
+    """Milliseconds per kernel family of one untimed pass (every launch bracketed by events)."""
+    torch.cuda.synchronize()
+    msa.profile_reset()
+    msa.profile_enable(True)
+    pf.run()
+    torch.cuda.synchronize()
+    msa.profile_enable(False)
+    fam = {}
+    for f in ("block_keys", "index_scores", "select_topk", "index_topk", "prefill_lists", "prefill_attn",
+              "prefill_combine"):
+        t, n = msa.profile_read(f)
+        if n:
+            fam[f] = round(t, 3)
+    msa.profile_reset()
+    return fam
+
+
 def end_to_end(args, dist, pf, x, T):
+    """The same step from pinned host buffers to pinned host buffers (Prefill.run_from_host: chunk
+    copies overlap the computation of other chunks)."""
     host = {k: v.cpu().pin_memory() for k, v in x.items() if k in ("q", "k", "v", "wq", "wk")}
     o_host = torch.empty(pf.o.shape, dtype=pf.o.dtype, pin_memory=True)
     lse_host = torch.empty(pf.lse.shape, dtype=pf.lse.dtype, pin_memory=True)
@@ -433,15 +464,12 @@ def end_to_end(args, dist, pf, x, T):
     d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * lse_host.element_size()
 
     def e2e_step():
-        for k2, t in host.items():
-            x[k2].copy_(t, non_blocking=True)
-        pf.run()
-        o_host.copy_(pf.o, non_blocking=True)
-        lse_host.copy_(pf.lse, non_blocking=True)
+        pf.run_from_host(host, o_host, lse_host)
 
     ms_e2e = timed(e2e_step, args.steps, 1, dist)
     return {"value": throughput(dist.world, T, args.steps, ms_e2e), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / args.steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / args.steps,
+            "overlap": "per-chunk query copies and output copies overlap other chunks' compute"}
 
 
 def workload_config(w, T: int, chunk: int, world: int) -> dict:
@@ -455,16 +483,16 @@ def workload_config(w, T: int, chunk: int, world: int) -> dict:
             "parallelism": f"dp{world} (one independent sequence per rank)"}
 
 
-def emit(args, dist, w, T, pf, value, ms_step, roofline, cpu_baseline, e2e, launches, clk, step_tflops, fam,
+def emit(args, dist, w, T, chunk, value, ms_step, roofline, cpu_baseline, e2e, launches, clk, step_tflops, fam,
          secondary):
     if dist.rank != 0:
         return
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(w, T, pf.chunk, dist.world),
+            "config": workload_config(w, T, chunk, dist.world),
             "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clk, "step_tflops_selected": step_tflops, "kernel_ms_per_step": fam,
+            "clocks": clk, "step_tflops_selected": step_tflops, "kernel_ms_one_step": fam,
             "secondary": secondary}
     print(json.dumps(line), flush=True)
 
@@ -539,8 +567,14 @@ def one_million(args, dist, pk):
     dc.prepare_keys()
     between = l2_flusher()
     ms = timed(dc.graph(), 20, 3, dist, between=between)
+    attn = graph_of(lambda: msa.msa_sparse_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.block_idx,
+                                                       dc.o, dc.lse, dc.workspace, dc.err))
+    a_ms = timed(attn.replay, 20, 3, dist, between=between) / 20
+    sel = decode_selected_bytes(dc)
     out["decode_1m"] = {"ms_per_step": ms / 20, "tokens_per_s": dist.world * wd.batch * 20 / (ms / 1000),
-                        "selected_bytes": decode_selected_bytes(dc), "graph": True, "l2": L2_NOTE}
+                        "attn_ms": a_ms, "selected_bytes": sel, "attn_gbs": sel / (a_ms / 1000) / 1e9,
+                        "hbm_frac": sel / (a_ms / 1000) / 1e9 / float(pk["hbm_gbs"]), "graph": True, "l2": L2_NOTE}
+    del attn
     ws = msa.msa_dense_attn_decode(dc.cfg, dc.shape, None, None, None, None, None, None)
     wsb = torch.empty(ws, dtype=torch.uint8, device="cuda")
     msd = timed(lambda: msa.msa_dense_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.o, dc.lse, wsb),

@@ -28,6 +28,7 @@ std::mutex g_prof_mu;
 std::atomic<bool> g_prof_on{false};
 std::vector<ProfRec> g_prof_recs;
 std::vector<cudaEvent_t> g_prof_pool;
+std::string g_prof_only;   // bracket only this family ("" = every family); guarded by g_prof_mu
 thread_local cudaEvent_t t_prof_open = nullptr;
 
 cudaEvent_t prof_event() {
@@ -216,9 +217,10 @@ void *decode_scratch_address() {
 }  // namespace
 
 namespace msa {
-void prof_begin(const char *, cudaStream_t st) {
+void prof_begin(const char *family, cudaStream_t st) {
     if (!g_prof_on.load(std::memory_order_relaxed)) return;
     std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (!g_prof_only.empty() && g_prof_only != family) return;
     t_prof_open = prof_event();
     if (t_prof_open) cudaEventRecord(t_prof_open, st);
 }
@@ -237,6 +239,11 @@ void prof_end(const char *family, cudaStream_t st) {
 extern "C" {
 
 void msa_profile_enable(int on) { g_prof_on.store(on != 0); }
+
+void msa_profile_only(const char *family) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_only = family ? family : "";
+}
 
 void msa_profile_reset(void) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
@@ -290,7 +297,9 @@ msa_status_t msa_index_scores(const msa_config_t *cfg, const msa_shape_t *shape,
     if (!aligned(q, 16) || !aligned(wq, 16) || !aligned(k_idx, 16) || !aligned(scores, 16) ||
         (k && (!aligned(k, 16) || !aligned(wk, 16))) || (q_idx_out && !aligned(q_idx_out, 16)))
         return MSA_ERR_INVALID_ARG;
-    if (row_begin < 0 || row_end < row_begin || row_end > shape->total_rows || kidx_from_block < 0)
+    if (row_begin < 0 || row_end < row_begin || row_end > shape->total_rows) return MSA_ERR_INVALID_ARG;
+    // a negative kidx_from_block is only MSA_KIDX_NEWEST_BLOCK, and only for a decode cache of keys
+    if (kidx_from_block < 0 && (kidx_from_block != MSA_KIDX_NEWEST_BLOCK || shape->mode != MSA_DECODE || !k))
         return MSA_ERR_INVALID_ARG;
     if (scores_row_stride < shape->max_blocks || scores_row_stride % 4) return MSA_ERR_INVALID_ARG;
     const Prob P = make_prob(cfg, shape, row_begin, row_end, nullptr);
@@ -322,9 +331,11 @@ msa_status_t msa_select_topk(const msa_config_t *cfg, const msa_shape_t *shape, 
     msa_status_t st = check_cfg(cfg);
     if (st != MSA_OK) return st;
     if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
-    if (!scores || !block_idx || !aligned(scores, 4) || !aligned(block_idx, 4)) return MSA_ERR_INVALID_ARG;
+    // long rows are copied 16 bytes at a time from the start of each score row (whole 16-byte
+    // chunks up to the row's candidate count, which stay inside a stride that is a multiple of 4)
+    if (!scores || !block_idx || !aligned(scores, 16) || !aligned(block_idx, 4)) return MSA_ERR_INVALID_ARG;
     if (row_begin < 0 || row_end < row_begin || row_end > shape->total_rows) return MSA_ERR_INVALID_ARG;
-    if (scores_row_stride < shape->max_blocks) return MSA_ERR_INVALID_ARG;
+    if (scores_row_stride < shape->max_blocks || scores_row_stride % 4) return MSA_ERR_INVALID_ARG;
     const Prob P = make_prob(cfg, shape, row_begin, row_end, err_flag);
     cudaError_t e = launch_select_topk(P, scores, scores_row_stride, block_idx, static_cast<cudaStream_t>(stream));
     return cuda_status(e, row_end > row_begin ? 1 : 0);

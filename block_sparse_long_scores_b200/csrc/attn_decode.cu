@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(NW * 32) decode_attn_kernel(Prob P, const __gr
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = blockIdx.z, g = blockIdx.y, cta = blockIdx.x, nct = gridDim.x;
     const int64_t bg = (int64_t)b * P.Hkv + g;
-    const int64_t len = P.seqlens[b];
+    const int64_t len = decode_len(P, b);
     const int64_t pos = len - 1;
     const int64_t i = pos / BLK;
     const bool dense = block_idx == nullptr;
@@ -469,12 +469,15 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
         // Entering a (b, g) row, the warp loads its block list once and sanitises it (out of range,
         // future or repeated -> -1, flagged); lane 0 then streams the row's blocks of this range.
         int cur_bg = -1;
+        int last_load[NS];                // lane 0: per stage, its latest item if that item loaded K/V
+#pragma unroll
+        for (int s = 0; s < NS; ++s) last_load[s] = -1;
         int bg = bg_first, a = a_first;   // item x0 + k is slot a of row bg
         for (int k = 0; k < n; ++k, a = (a + 1 == k_tot) ? 0 : a + 1, bg += (a == 0)) {
             if (bg != cur_bg) {
                 __syncwarp();
                 const int b = bg / P.Hkv;
-                const int64_t i = ((int64_t)P.seqlens[b] - 1) / BLK;
+                const int64_t i = (decode_len(P, b) - 1) / BLK;
                 const int32_t *row = block_idx + (int64_t)bg * k_tot;
                 bool canon = true;
                 int bad = 0;
@@ -514,6 +517,9 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                 if (fail) {
                 } else if (j >= 0) {
                     mbar_arrive_expect_tx(&S.full[s], 2 * DC * SM::KV_CHUNK);
+#pragma unroll
+                    for (int t = 0; t < NS; ++t)
+                        if (t == s) last_load[t] = k;
                     const int row0 = (int)((int64_t)bg * P.Lmax + (int64_t)j * BLK);
 #pragma unroll
                     for (int cc = 0; cc < DC; ++cc) {
@@ -522,9 +528,19 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                     }
                 } else {
                     mbar_arrive(&S.full[s]);   // nothing to load: the slot is skipped
+#pragma unroll
+                    for (int t = 0; t < NS; ++t)   // the stage's earlier load was consumed before this
+                        if (t == s) last_load[t] = -1;
                 }
             }
             if (__any_sync(0xffffffffu, fail != 0)) break;
+        }
+        // after a wait ran out, the loads already issued must land before the CTA's shared memory
+        // is released: wait (bounded) for the completion of each stage's latest load
+        if (lane == 0 && fail) {
+#pragma unroll
+            for (int t = 0; t < NS; ++t)
+                if (last_load[t] >= 0) mbar_wait(&S.full[t], (last_load[t] / NS) & 1);
         }
     } else {
         // ------------------------------------------------------------------ consumers
@@ -605,7 +621,7 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
         int loc_blk = 0, loc_lim = 0;   // the current row's local block and its last valid key
         auto load_q = [&](int bg) {
             const int b = bg / P.Hkv, g = bg - b * P.Hkv;
-            const int64_t pos = (int64_t)P.seqlens[b] - 1;
+            const int64_t pos = decode_len(P, b) - 1;
             loc_blk = (int)(pos / BLK);
             loc_lim = (int)(pos - (int64_t)loc_blk * BLK);
             const int r0 = lane >> 2, r1 = r0 + 8;

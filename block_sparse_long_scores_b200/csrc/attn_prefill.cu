@@ -325,6 +325,9 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
         int ent = (nt > 0 && lane < td.z) ? W.entries[td.y + lane] : 0;
         int64_t cur_list = -1;
         int kv_uses = 0;
+        int kv_last[A::NKV];   // per K/V stage: the use number of its latest load (-1: none)
+#pragma unroll
+        for (int s2 = 0; s2 < A::NKV; ++s2) kv_last[s2] = -1;
         for (int i = 0; i < nt; ++i) {
             // descriptor and entries of tile i+1 (issued now, consumed next iteration)
             int4 td_n = make_int4(-1, 0, 0, 0);
@@ -372,6 +375,9 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
                 if (!__all_sync(0xffffffffu, ok)) break;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&S.kv_full[kvs], 2 * A::KV_STAGE);
+#pragma unroll
+                    for (int s2 = 0; s2 < A::NKV; ++s2)
+                        if (s2 == kvs) kv_last[s2] = kv_uses - 1;
                     const int row0 = (int)(s0 + j * BLK);
 #pragma unroll
                     for (int cc = 0; cc < A::DC; ++cc) {
@@ -382,6 +388,12 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
             }
             td = td_n;
             ent = ent_n;
+        }
+        // after a wait ran out, K/V loads already issued must land before the CTA exits
+        if (lane == 0 && *(volatile int *)&S.fail) {
+#pragma unroll
+            for (int s2 = 0; s2 < A::NKV; ++s2)
+                if (kv_last[s2] >= 0) mbar_wait(&S.kv_full[s2], (kv_last[s2] / A::NKV) & 1);
         }
     } else if (warp == 2 || warp == 3) {
         // ------------------------------------------------------------------ query gather (warps 2, 3)
@@ -423,6 +435,7 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
             }
             cp_async_arrive_noinc(&S.q_full[qs]);
         }
+        cp_async_wait<0>();   // no gather copy may still be in flight when the CTA exits
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {

@@ -49,6 +49,17 @@ __device__ __forceinline__ int seq_of_row(const int32_t *cu, int batch, int64_t 
     return lo;
 }
 
+// Cache length of decode sequence b (it counts the new token), clamped to [1, Lmax] so that no
+// kernel indexes past the cache; a length outside that range is flagged as a shape error.
+__device__ __forceinline__ int64_t decode_len(const Prob &P, int b) {
+    int64_t L = P.seqlens[b];
+    if (L < 1 || L > P.Lmax) {
+        report(P.err, kErrShape);
+        L = L < 1 ? 1 : P.Lmax;
+    }
+    return L;
+}
+
 // Row geometry: sequence b, first row of the sequence, its length, in-sequence position.
 struct RowGeo {
     int b;
@@ -67,7 +78,7 @@ __device__ __forceinline__ RowGeo row_geo(const Prob &P, int64_t row) {
     } else {
         g.b = (int)row;
         g.s0 = 0;
-        g.len = P.seqlens[row];
+        g.len = decode_len(P, (int)row);
         g.pos = g.len - 1;
     }
     return g;

@@ -17,7 +17,8 @@ namespace msa {
 
 // ------------------------------------------------------------------------------- block keys
 
-// One CTA per block (prefill: global block number; decode: (b, j)); 256 threads.
+// One CTA per block (prefill: global block number; decode: (b, j), or with from_block < 0 one
+// CTA per sequence b for its newest token's block j = (seqlens[b] - 1) / B); 256 threads.
 // smem: kbar [Hkv][D] fp32, W_k [D][d] bf16.
 __global__ void __launch_bounds__(256) block_keys_kernel(Prob P, const __nv_bfloat16 *__restrict__ K,
                                                          const __nv_bfloat16 *__restrict__ Wk,
@@ -27,6 +28,8 @@ __global__ void __launch_bounds__(256) block_keys_kernel(Prob P, const __nv_bflo
     __nv_bfloat16 *Ws = reinterpret_cast<__nv_bfloat16 *>(smem_raw + sizeof(float) * P.Hkv * P.D);
     const int tid = threadIdx.x;
     const int D = P.D, d = P.d, Hkv = P.Hkv, B = P.B;
+    griddep_wait();     // lengths and cache rows may come from earlier work in the stream
+    griddep_launch();
 
     int b;
     int64_t j, len, nblk;
@@ -35,13 +38,18 @@ __global__ void __launch_bounds__(256) block_keys_kernel(Prob P, const __nv_bflo
         b = seq_of_row(P.cu_blocks, P.batch, gb);
         j = gb - P.cu_blocks[b];
         len = (int64_t)P.cu_seqlens[b + 1] - P.cu_seqlens[b];
+    } else if (from_block < 0) {
+        b = (int)blockIdx.x;
+        len = decode_len(P, b);
+        j = (len - 1) / B;
+        from_block = 0;
     } else {
         b = (int)(blockIdx.x / P.max_blocks);
         j = blockIdx.x % P.max_blocks;
-        len = P.seqlens[b];
+        len = decode_len(P, b);
     }
     nblk = (len + B - 1) / B;
-    if (j < from_block || j >= nblk) return;
+    if (j < from_block || j >= nblk || j >= P.max_blocks) return;
     const int64_t t_first = j * B;
     const int n = (int)lmin(B, len - t_first);
 
@@ -298,7 +306,7 @@ __global__ void __launch_bounds__(256, 4) index_scores_decode_kernel(Prob P, con
     griddep_launch();
     const int64_t r = P.row_begin + blockIdx.z;
     const int b = (int)r;
-    const int64_t i = ((int64_t)P.seqlens[b] - 1) / P.B;
+    const int64_t i = (decode_len(P, b) - 1) / P.B;
     const int64_t j0 = (int64_t)blockIdx.x * kDecKeysPerCta;
     const bool write_q = blockIdx.x == 0 && qidx_out;
     if (j0 >= i && !write_q) return;
@@ -362,7 +370,8 @@ __global__ void __launch_bounds__(256, 4) index_scores_decode_kernel(Prob P, con
 
 cudaError_t launch_block_keys(const Prob &P, const void *K, const void *Wk, void *kidx, int64_t from_block,
                               cudaStream_t st) {
-    const int64_t nctas = P.mode == 0 ? P.total_blocks : (int64_t)P.batch * P.max_blocks;
+    const int64_t nctas = P.mode == 0 ? P.total_blocks
+                                      : (from_block < 0 ? (int64_t)P.batch : (int64_t)P.batch * P.max_blocks);
     if (nctas == 0) return cudaSuccess;
     const size_t smem = sizeof(float) * P.Hkv * P.D + sizeof(__nv_bfloat16) * P.D * P.d;
     if (smem > 48 * 1024) {
@@ -370,9 +379,8 @@ cudaError_t launch_block_keys(const Prob &P, const void *K, const void *Wk, void
         if (e != cudaSuccess) return e;
     }
     ProfScope prof("block_keys", st);
-    block_keys_kernel<<<(unsigned)nctas, 256, smem, st>>>(P, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)Wk,
-                                                         (__nv_bfloat16 *)kidx, from_block);
-    return cudaGetLastError();
+    return launch_pdl(block_keys_kernel, dim3((unsigned)nctas), dim3(256), smem, st, P, (const __nv_bfloat16 *)K,
+                      (const __nv_bfloat16 *)Wk, (__nv_bfloat16 *)kidx, from_block);
 }
 
 size_t index_tc_smem() { return sizeof(IdxSmem) + 1024; }

@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libmsa_b200.so")
 
 MSA_PREFILL = 0
 MSA_DECODE = 1
+MSA_KIDX_NEWEST_BLOCK = -1    # kidx_from_block: only each decode sequence's newest block
 
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_WORKSPACE",
           4: "MSA_ERR_CUDA"}
@@ -28,7 +29,7 @@ DERR = {1: "BLOCK_RANGE", 2: "DUPLICATE", 4: "NAN_SCORE", 8: "TIMEOUT", 16: "SHA
 EXPORTED = ("msa_index_scores", "msa_select_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
             "msa_dense_attn_prefill", "msa_dense_attn_decode", "msa_status_string", "msa_version",
             "msa_launch_count", "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
-            "msa_sparse_attn_decode_noalloc")
+            "msa_sparse_attn_decode_noalloc", "msa_profile_only")
 
 
 class MSAError(RuntimeError):
@@ -88,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.msa_launch_count.restype = I64
         L.msa_profile_enable.argtypes = [ctypes.c_int]
         L.msa_profile_enable.restype = None
+        L.msa_profile_only.argtypes = [ctypes.c_char_p]
+        L.msa_profile_only.restype = None
         L.msa_profile_reset.argtypes = []
         L.msa_profile_reset.restype = None
         L.msa_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64)]
@@ -218,6 +221,11 @@ def launch_count() -> int:
 
 def profile_enable(on: bool = True):
     lib().msa_profile_enable(1 if on else 0)
+
+
+def profile_only(family: str | None = None):
+    """Bracket only this kernel family while profiling is enabled (None: every family)."""
+    lib().msa_profile_only(family.encode() if family else None)
 
 
 def profile_reset():

@@ -69,6 +69,45 @@ class Prefill:
             self.attend(r0, r1)
         return self.o, self.lse
 
+    def run_from_host(self, host: dict, o_host: torch.Tensor, lse_host: torch.Tensor | None = None):
+        """One pass of the hot path whose inputs start in (pinned) host memory and whose outputs end
+        there.  K, V, W_q and W_k are copied first; then each row chunk's queries are copied on a
+        copy stream while the previous chunk computes, and each chunk's O (and lse) rows go back on
+        a second copy stream as soon as the chunk is done.  Returns once everything is enqueued; the
+        caller's current stream waits for the last copy back."""
+        cur = torch.cuda.current_stream()
+        if not hasattr(self, "_h2d"):
+            self._h2d, self._d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        h2d, d2h = self._h2d, self._d2h
+        x = self.x
+        h2d.wait_stream(cur)        # the previous pass may still read the device inputs
+        d2h.wait_stream(cur)
+        ready = []
+        with torch.cuda.stream(h2d):
+            for name in ("k", "v", "wq", "wk"):
+                x[name].copy_(host[name], non_blocking=True)
+            for r0, r1 in self.chunks():
+                x["q"][r0:r1].copy_(host["q"][r0:r1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(h2d)
+                ready.append(ev)
+        first = True
+        for c, (r0, r1) in enumerate(self.chunks()):
+            cur.wait_event(ready[c])
+            self.index(r0, r1, compute_keys=first)
+            first = False
+            self.select(r0, r1)
+            self.attend(r0, r1)
+            done = torch.cuda.Event()
+            done.record(cur)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                o_host[r0:r1].copy_(self.o[r0:r1], non_blocking=True)
+                if lse_host is not None and self.lse is not None:
+                    lse_host[r0:r1].copy_(self.lse[r0:r1], non_blocking=True)
+        cur.wait_stream(d2h)
+        return o_host, lse_host
+
 
 class Decode:
     """One decode step of workload `w`: the new token of every sequence against its cache."""
@@ -101,27 +140,36 @@ class Decode:
                              self.scores, self.stride)
         self.keys_ready = True
 
-    def graph(self):
-        """Capture one decode step (index scores -> selection -> attention) in a CUDA graph and
-        return its replay function.  Every replay reads the same input tensors (refresh them in
-        place between steps) and writes the same outputs; the kernels inside are chained with
+    def graph(self, q_idx_out=None):
+        """Capture one decode step (newest block key -> index scores -> selection -> attention) in
+        a CUDA graph and return its replay function.  Every replay reads the same input tensors
+        (refresh them in place between steps: new queries, the new tokens' K/V in the cache, the
+        advanced seqlens) and writes the same outputs; the kernels inside are chained with
         programmatic dependent launch."""
         if not self.keys_ready:
             self.prepare_keys()
-        self.run()                 # first call: per-kernel attributes set outside the capture
+        self.run(q_idx_out)        # first call: per-kernel attributes set outside the capture
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            self.run()
+            self.run(q_idx_out)
         self._graph = g
         return g.replay
 
     def run(self, q_idx_out=None):
+        """One decode step.  Unless the block keys were given, the step first refreshes the key of
+        each sequence's newest block (the block the new token belongs to), so a loop that appends
+        one token per sequence per step -- writing its K/V into the cache and advancing `seqlens` in
+        place -- keeps the key cache current, also under CUDA graph replay."""
         x = self.x
         if not self.keys_ready:
             self.prepare_keys()
-        msa.msa_index_scores(self.cfg, self.shape, x["q"], None, x["wq"], None, self.k_idx, 0, 0, self.w.batch,
-                             self.scores, self.stride, q_idx_out)
+        if self.given_kidx:
+            msa.msa_index_scores(self.cfg, self.shape, x["q"], None, x["wq"], None, self.k_idx, 0, 0,
+                                 self.w.batch, self.scores, self.stride, q_idx_out)
+        else:
+            msa.msa_index_scores(self.cfg, self.shape, x["q"], x["k"], x["wq"], x["wk"], self.k_idx,
+                                 msa.MSA_KIDX_NEWEST_BLOCK, 0, self.w.batch, self.scores, self.stride, q_idx_out)
         msa.msa_select_topk(self.cfg, self.shape, self.scores, self.stride, 0, self.w.batch, self.block_idx, self.err)
         msa.msa_sparse_attn_decode(self.cfg, self.shape, x["q"], x["k"], x["v"], self.block_idx, self.o, self.lse,
                                    self.workspace, self.err)

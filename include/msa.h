@@ -50,8 +50,9 @@
  *            returns MSA_ERR_INVALID_ARG / MSA_ERR_UNSUPPORTED and launches nothing.  A CUDA
  *            launch failure returns MSA_ERR_CUDA.  Bad *data* found on the device (a block
  *            number out of range or in the future, a repeated block, a NaN score, a wait that
- *            ran out of time) is skipped and reported by OR-ing an MSA_DERR_* bit into
- *            *err_flag (device int32, nullable); kernels never trap.
+ *            ran out of time, a decode length outside [1, Lmax], which is clamped into that
+ *            range) is skipped and reported by OR-ing an MSA_DERR_* bit into *err_flag (device
+ *            int32, nullable); kernels never trap.
  * Workspace. Calls that need scratch take (workspace, workspace_bytes).  With workspace == NULL
  *            the call only writes the required size to *workspace_bytes and returns MSA_OK;
  *            otherwise *workspace_bytes must be at least that size (else MSA_ERR_WORKSPACE).
@@ -72,6 +73,9 @@ extern "C" {
 
 #define MSA_PREFILL 0
 #define MSA_DECODE 1
+
+/* kidx_from_block value of msa_index_scores: only the block of each sequence's newest token. */
+#define MSA_KIDX_NEWEST_BLOCK (-1)
 
 typedef enum {
     MSA_OK = 0,
@@ -119,6 +123,11 @@ typedef struct {
  *  1. If k != NULL, block keys are (re)computed for every block j >= kidx_from_block of every
  *     sequence (j counted within its sequence):
  *        k_idx[j, g] = bf16( (mean over the valid tokens t of block j of K[t, g, :]) . W_k ).
+ *     Decode only: kidx_from_block = MSA_KIDX_NEWEST_BLOCK recomputes just the block holding each
+ *     sequence's newest token, j = (seqlens[b] - 1) / B.  A decode loop that appends one token per
+ *     sequence per step and passes this every step keeps its key cache current: the newest block
+ *     is never scored in its own step (it is the local block), and once its last token has arrived
+ *     its key is the mean of the whole block by the time the next step scores it.
  *     If k == NULL, k_idx is read as given (e.g. a decode cache of block keys kept by the caller,
  *     or keys supplied directly); wk may then be NULL.
  *  2. For every row r in [row_begin, row_end) and kv head g:
@@ -148,7 +157,8 @@ msa_status_t msa_index_scores(const msa_config_t *cfg, const msa_shape_t *shape,
  *    block_idx[r - row_begin, g, :] = ascending( picks + {i} + ({0} if use_sink and i > 0) ),
  *            padded with -1 to k_tot = n_topk + 1 + use_sink entries.
  *  A NaN score is skipped (never picked) and raises MSA_DERR_NAN_SCORE in *err_flag (nullable).
- *  scores: as written by msa_index_scores for the same row range.
+ *  scores: as written by msa_index_scores for the same row range; the same rules hold (16-byte
+ *  aligned base, scores_row_stride >= max_blocks and a multiple of 4), else MSA_ERR_INVALID_ARG.
  */
 msa_status_t msa_select_topk(const msa_config_t *cfg, const msa_shape_t *shape,
                              const float *scores, int64_t scores_row_stride,
@@ -256,8 +266,11 @@ int64_t msa_launch_count(void);
  * recorded on the caller's stream.  msa_profile_read waits for the recorded events and returns the
  * summed milliseconds and the number of bracketed launches of one family (NULL: all families);
  * msa_profile_reset forgets them.  Disabled by default; costs two event records per launch.
+ * msa_profile_only restricts the bracketing to one family (NULL or "": every family), so that one
+ * kernel can be timed inside a measured region without events around the others.
  */
 void msa_profile_enable(int on);
+void msa_profile_only(const char *family);
 void msa_profile_reset(void);
 int32_t msa_profile_read(const char *family, double *total_ms, int64_t *launches);
 

@@ -130,6 +130,39 @@ def test_index_scores_rejects_bad_stride(L):
         assert rc == 1
 
 
+def test_newest_block_key_mode_is_decode_only(L):
+    # kidx_from_block = MSA_KIDX_NEWEST_BLOCK (-1) needs decode mode and K; other negatives are errors
+    cfg = _cfg()
+    fake = ctypes.c_void_p(0x100000)
+    pre = _prefill_shape()
+    rc = L.msa_index_scores(ctypes.byref(cfg), ctypes.byref(pre), fake, fake, fake, fake, fake,
+                            msa.MSA_KIDX_NEWEST_BLOCK, 0, 10, fake, 2048, None, None)
+    assert rc == 1
+    dec = _decode_shape(4, 4096)
+    rc = L.msa_index_scores(ctypes.byref(cfg), ctypes.byref(dec), fake, None, fake, None, fake,
+                            msa.MSA_KIDX_NEWEST_BLOCK, 0, 4, fake, 64, None, None)
+    assert rc == 1                                                # no K to compute keys from
+    rc = L.msa_index_scores(ctypes.byref(cfg), ctypes.byref(dec), fake, fake, fake, fake, fake, -2, 0, 4, fake, 64,
+                            None, None)
+    assert rc == 1
+
+
+def test_select_topk_rejects_misaligned_scores_and_bad_stride(L):
+    # long score rows are copied 16 bytes at a time: the base must be 16-byte aligned and the row
+    # stride a multiple of 4 floats (at least max_blocks), as for msa_index_scores
+    cfg, shape = _cfg(), _prefill_shape()
+    fake = ctypes.c_void_p(0x100000)
+    cases = [(ctypes.c_void_p(0x100004), 2048),   # 4-byte aligned only
+             (fake, 2047),                        # below max_blocks
+             (fake, 2050)]                        # not a multiple of 4
+    for scores, stride in cases:
+        rc = L.msa_select_topk(ctypes.byref(cfg), ctypes.byref(shape), scores, stride, 0, 10, fake, None, None)
+        assert rc == 1
+    # a valid call on an empty row range launches nothing and succeeds
+    rc = L.msa_select_topk(ctypes.byref(cfg), ctypes.byref(shape), fake, 2048, 5, 5, fake, None, None)
+    assert rc == 0
+
+
 def _decode_shape(batch, Lmax, B=64):
     return msa.Shape(msa.MSA_DECODE, batch, None, None, 0x10000, batch, 0, Lmax, (Lmax + B - 1) // B)
 

@@ -66,7 +66,7 @@ def test_emitted_line_carries_the_contract_keys(capsys):
     e2e = {"value": 1.5e6, "unit": "tokens/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 1}
     clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
     bench.emit(SimpleNamespace(steps=5, warmup=3), SimpleNamespace(rank=0, world=1), w, 131072,
-               SimpleNamespace(chunk=16384), 3.1e6, 41.5, roofline, cpu, e2e, 325, clk, 213.0, {}, {})
+               16384, 3.1e6, 41.5, roofline, cpu, e2e, 325, clk, 213.0, {}, {})
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     for key, typ in [("metric", str), ("value", float), ("unit", str), ("n_gpus", int), ("steps", int),
                      ("warmup", int), ("ms_per_step", float), ("higher_is_better", bool), ("scaling", str),
@@ -80,7 +80,7 @@ def test_emitted_line_carries_the_contract_keys(capsys):
     # the ragged workload has no sink and unequal lengths
     wr = WORKLOADS["ragged_prefill"]
     bench.emit(SimpleNamespace(steps=1, warmup=1), SimpleNamespace(rank=0, world=1), wr, sum(wr.seqlens),
-               SimpleNamespace(chunk=16384), 1.0, 1.0, roofline, None, None, 1, clk, 1.0, {}, {})
+               16384, 1.0, 1.0, roofline, None, None, 1, clk, 1.0, {}, {})
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert "+ sink" not in line["config"]["workload"] and "(ragged)" in line["config"]["workload"]
 

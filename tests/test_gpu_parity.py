@@ -97,6 +97,23 @@ def test_prefill_128k_shape_small_multichunk():
     _prefill_full_check(w, x, chunk_rows=2048)
 
 
+@pytest.mark.parametrize("gain", [11.3137, 45.2548])
+def test_prefill_128k_shape_sharp_logits(gain):
+    # the headline kernel instantiation (G 8, D 128, B 64) with q, k ~ N(0,1) and 4x that: the
+    # logits reach several units, so the running max and the partials' rescaling are exercised
+    w = scaled_down(WORKLOADS["prefill_128k"], (6000,))
+    x = make_inputs(w, device=DEV, seed=31, logit_gain=gain)
+    _prefill_full_check(w, x, chunk_rows=2048)
+
+
+@pytest.mark.parametrize("gain", [8.0, 32.0])
+def test_ragged_shape_sharp_logits(gain):
+    # the ragged instantiation (G 8, D 64, B 128) with q, k ~ N(0,1) and 4x that
+    w = scaled_down(WORKLOADS["ragged_prefill"], (130, 3000, 64, 2100))
+    x = make_inputs(w, device=DEV, seed=32, logit_gain=gain)
+    _prefill_full_check(w, x, chunk_rows=1500)
+
+
 def test_ragged_prefill_small_with_ties():
     # ragged workload shape (64/8 heads, D 64, B 128, k 32, discrete index keys -> exact ties)
     w = scaled_down(WORKLOADS["ragged_prefill"], (1, 130, 1000, 64, 2900, 129, 700))
@@ -197,6 +214,11 @@ def _decode_check(w, x):
     qidx = torch.empty(w.batch, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV)
     dc.run(q_idx_out=qidx)
     torch.cuda.synchronize()
+    return _decode_compare(w, x, dc, qidx)
+
+
+def _decode_compare(w, x, dc, qidx):
+    """One decode step's outputs (key cache, q_idx, scores, selection, O, lse) against the oracle."""
     assert int(dc.err.item()) == 0
     xc = cpu(x)
     sh = oracle_shape(w, xc)
@@ -284,6 +306,53 @@ def test_decode_graph_replay_recomputes():
         assert torch.equal(o_graph, dc.o) and torch.equal(lse_graph, dc.lse)
 
 
+def test_decode_graph_appends_tokens_across_block_boundaries():
+    # a decode loop on one captured step: before each replay every sequence gains a token (its K/V
+    # are already in the cache tensor; seqlens advances in place) and new queries arrive.  The step
+    # refreshes the key of each sequence's newest block, so blocks that completed in earlier steps
+    # (at lengths 64, 128, 192) are scored with the mean of all their tokens
+    Lmax = 320
+    lens0 = np.array([62, 126, 190, 1, 255], np.int32)
+    w = scaled_down(WORKLOADS["decode_128k"], (Lmax,) * len(lens0)).with_(n_topk=2)
+    x = make_inputs(w, device=DEV, seed=27)
+    x["seqlens"].copy_(torch.as_tensor(lens0))
+    w = w.with_(seqlens=tuple(int(v) for v in lens0))   # host view of the starting lengths
+    dc = Decode(w, x)
+    qidx = torch.empty(w.batch, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV)
+    step = dc.graph(q_idx_out=qidx)
+    g = torch.Generator(device="cpu").manual_seed(28)
+    for t in range(5):
+        if t:
+            x["seqlens"].add_(1)
+            x["q"].copy_(torch.randn(x["q"].shape, generator=g).to(x["q"].dtype))
+        step()
+        torch.cuda.synchronize()
+        lens = lens0 + t
+        assert np.array_equal(x["seqlens"].cpu().numpy(), lens)
+        _decode_compare(w.with_(seqlens=tuple(int(v) for v in lens)), x, dc, qidx)
+
+
+def test_decode_lengths_beyond_the_cache_are_clamped_and_flagged():
+    # a seqlens entry above the cache capacity (or below 1) is a shape error: flagged, clamped
+    w = scaled_down(WORKLOADS["decode_128k"], (300, 200))
+    x = make_inputs(w, device=DEV, seed=29)
+    dc = Decode(w, x)
+    dc.run()
+    torch.cuda.synchronize()
+    assert int(dc.err.item()) == 0
+    x["seqlens"][1] = 100000
+    dc.run()
+    torch.cuda.synchronize()
+    assert int(dc.err.item()) & 16
+    o_clamped = dc.o[1].clone()
+    x["seqlens"][1] = 300
+    dc.err.zero_()
+    dc.run()
+    torch.cuda.synchronize()
+    assert int(dc.err.item()) == 0
+    assert torch.equal(o_clamped, dc.o[1])
+
+
 def test_decode_bad_and_unordered_block_ids_are_flagged_and_skipped():
     # the decode kernel sanitises each block list once per CTA: out-of-range ids and repeats are
     # skipped and flagged, any order is accepted (the selection is a set)
@@ -343,7 +412,7 @@ def test_dense_decode_matches_oracle():
 def test_prefill_128k_full_size_sampled():
     w = WORKLOADS["prefill_128k"]
     x = make_inputs(w, device=DEV)
-    rows = sample_rows(w, 256)
+    rows = sample_rows(w, 4096)
     _prefill_full_check(w, x, chunk_rows=16384, rows=rows, check_keys=True)
 
 
@@ -418,7 +487,29 @@ def test_ragged_prefill_full_size_sampled():
     _prefill_sampled_check(w, x, sample_rows(w, 4096, seed=2), chunk_rows=16384)
 
 
-def _decode_sampled_check(w, x):
+def _check_decode_key_cache(w, x, dc, n_blocks, seed):
+    """The GPU's block-key cache against the oracle on sampled blocks: their K rows are gathered
+    into a compact host cache (a block key depends only on its own rows), so the oracle reads only
+    the sampled blocks.  Every sampled block is complete."""
+    rng = np.random.default_rng(seed)
+    lens = x["seqlens"].cpu().numpy()
+    full = [int(l) // w.B for l in lens]
+    ns = min(n_blocks, min(full))
+    picks = [np.sort(rng.choice(full[b], size=ns, replace=False)) for b in range(w.batch)]
+    kc = torch.empty((w.batch, w.Hkv, ns * w.B, w.D), dtype=x["k"].dtype)
+    for b in range(w.batch):
+        rows = (torch.as_tensor(picks[b], device=x["k"].device).view(-1, 1) * w.B +
+                torch.arange(w.B, device=x["k"].device).view(1, -1)).reshape(-1)
+        kc[b] = x["k"][b][:, rows].cpu()
+    sh = orc.decode_shape(np.full(w.batch, ns * w.B, np.int32), ns * w.B, ns, w.Hq, w.Hkv, w.D, w.B, w.d,
+                          w.n_topk, w.use_sink)
+    _, khat = orc.block_keys(sh, kc, x["wk"].cpu())
+    gpu = _bits(dc.k_idx)
+    got = np.stack([gpu[b][:, picks[b]] for b in range(w.batch)])
+    check_bf16_near(got, khat[:, :, :ns], "k_idx (sampled cache blocks)")
+
+
+def _decode_sampled_check(w, x, key_blocks=0):
     dc = Decode(w, x)
     qidx = torch.empty(w.batch, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV)
     dc.run(q_idx_out=qidx)
@@ -444,15 +535,25 @@ def _decode_sampled_check(w, x):
     assert np.array_equal(sel, orc.select_topk_f32(sh, S_gpu, rows))
     O_ref, L_ref = orc.sparse_attn(sh, xc["q"], xc["k"], xc["v"], sel, rows)
     check_attention(dc.o.float().cpu().numpy(), O_ref, dc.lse.cpu().numpy(), L_ref)
+    if key_blocks:
+        _check_decode_key_cache(w, x, dc, key_blocks, seed=7)
 
 
 @pytest.mark.slow
-def test_decode_1m_full_length():
-    # the 1M decode workload's length and selection (16384 blocks, 128 picks + sink + local) with 2
-    # of its 8 sequences, which keeps the host side small
-    w = WORKLOADS["decode_1m"].with_(seqlens=(1 << 20, (1 << 20) - 37))
+def test_decode_1m_full_size():
+    # the 1M decode workload as benchmarked: 8 sequences of 2^20 tokens, 128 picks + sink + local;
+    # the host copies hold only the selected blocks (the rest of each host tensor is never touched)
+    w = WORKLOADS["decode_1m"]
     x = make_inputs(w, device=DEV, seed=3)
-    _decode_sampled_check(w, x)
+    _decode_sampled_check(w, x, key_blocks=512)
+
+
+@pytest.mark.slow
+def test_decode_1m_length_with_partial_last_block():
+    # a 1M-long cache whose last block is partial (its local block holds 27 of 64 keys)
+    w = WORKLOADS["decode_1m"].with_(seqlens=(1 << 20, (1 << 20) - 37))
+    x = make_inputs(w, device=DEV, seed=5)
+    _decode_sampled_check(w, x, key_blocks=256)
 
 
 @pytest.mark.slow

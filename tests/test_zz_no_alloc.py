@@ -4,7 +4,8 @@ Some callers cannot pass the library a workspace -- their device memory belongs 
 allocator, or their decode step must not call the CUDA allocator -- so the library offers a
 decode call whose scratch is a fixed device array it declares itself.  This file checks, through
 the C ABI, that the call gives the same output as the workspace-taking msa_sparse_attn_decode
-(within the parity tolerances) on two calls in a row, since every call reuses the same scratch.
+(within the parity tolerances) on two calls in a row, since every call reuses the same scratch,
+and that both match the fp64 oracle on the same selection.
 It is named to be collected last, and works in a fresh process (where the first call performs
 the one-time address look-up) as well as after the other tests.
 """
@@ -15,7 +16,8 @@ import torch
 from block_sparse_long_scores_b200 import msa
 from block_sparse_long_scores_b200.pipeline import Decode
 from block_sparse_long_scores_b200.workloads import WORKLOADS, make_inputs, scaled_down
-from tests.parity_helpers import check_attention
+from oracle import oracle as orc
+from tests.parity_helpers import check_attention, cpu, oracle_shape
 
 pytestmark = pytest.mark.gpu
 
@@ -33,6 +35,10 @@ def test_noalloc_decode_matches_workspace_decode_twice():
     w, x, dc = _decode_inputs(11)
     ref_o = dc.o.double().cpu().numpy()
     ref_lse = dc.lse.double().cpu().numpy()
+    xc = cpu(x)
+    O_orc, L_orc = orc.sparse_attn(oracle_shape(w, xc), xc["q"], xc["k"], xc["v"], dc.block_idx.cpu().numpy(),
+                                   np.arange(w.batch))
+    check_attention(ref_o, O_orc, ref_lse, L_orc)
     for _ in range(2):
         o = torch.full_like(dc.o, float("nan"))
         lse = torch.full_like(dc.lse, float("nan"))
@@ -41,6 +47,7 @@ def test_noalloc_decode_matches_workspace_decode_twice():
         torch.cuda.synchronize()
         assert int(err.item()) == 0
         check_attention(o.float().cpu().numpy(), ref_o, lse.cpu().numpy(), ref_lse)
+        check_attention(o.float().cpu().numpy(), O_orc, lse.cpu().numpy(), L_orc)
 
 
 def test_noalloc_decode_second_problem_after_first():
