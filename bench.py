@@ -56,6 +56,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample budget")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the 1M-token and ragged workloads")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense GQA baselines")
     ap.add_argument("--seq-len", type=int, default=0, help="scaled-down sequence (profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -504,14 +505,15 @@ def secondary_measurements(args, dist, pf, x, sparse_ms, pk):
 
     out = {}
     # dense causal GQA prefill over the same 128K sequence
-    od = torch.empty_like(pf.o)
-    ld = torch.empty_like(pf.lse)
-    T = pf.shape.total_rows
-    ms_dense = timed(lambda: msa.msa_dense_attn_prefill(pf.cfg, pf.shape, x["q"], x["k"], x["v"], 0, T, od, ld),
-                     1, 1, dist)
-    out["dense_prefill_128k"] = {"ms": ms_dense, "tflops": dense_flops(pf.w) / (ms_dense / 1000) / 1e12,
-                                 "speedup_of_sparse_step": ms_dense / sparse_ms}
-    del od, ld
+    if not args.no_dense:
+        od = torch.empty_like(pf.o)
+        ld = torch.empty_like(pf.lse)
+        T = pf.shape.total_rows
+        ms_dense = timed(lambda: msa.msa_dense_attn_prefill(pf.cfg, pf.shape, x["q"], x["k"], x["v"], 0, T, od, ld),
+                         1, 1, dist)
+        out["dense_prefill_128k"] = {"ms": ms_dense, "tflops": dense_flops(pf.w) / (ms_dense / 1000) / 1e12,
+                                     "speedup_of_sparse_step": ms_dense / sparse_ms}
+        del od, ld
     # decode at 128K: batch 32, each step replayed from a CUDA graph, L2 flushed between steps
     wd = WORKLOADS["decode_128k"]
     xd = make_inputs(wd, device="cuda", seed=100 + dist.rank)
@@ -529,14 +531,16 @@ def secondary_measurements(args, dist, pf, x, sparse_ms, pk):
                           "attn_ms": a_ms_launch, "selected_bytes": sel_bytes, "attn_gbs": gbs,
                           "hbm_frac": gbs / float(pk["hbm_gbs"]), "graph": True, "l2": L2_NOTE}
     del attn
-    ws = msa.msa_dense_attn_decode(dc.cfg, dc.shape, None, None, None, None, None, None)
-    wsb = torch.empty(ws, dtype=torch.uint8, device="cuda")
-    msd = timed(lambda: msa.msa_dense_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.o, dc.lse, wsb),
-                5, 2, dist, between=between)
-    dense_bytes = sum(wd.seqlens) * wd.Hkv * wd.D * 4
-    out["dense_decode_128k"] = {"ms": msd / 5, "gbs": dense_bytes / (msd / 5 / 1000) / 1e9,
-                                "speedup_of_sparse_attn": (msd / 5) / a_ms_launch}
-    del xd, dc, wsb
+    if not args.no_dense:
+        ws = msa.msa_dense_attn_decode(dc.cfg, dc.shape, None, None, None, None, None, None)
+        wsb = torch.empty(ws, dtype=torch.uint8, device="cuda")
+        msd = timed(lambda: msa.msa_dense_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.o, dc.lse,
+                                                      wsb), 5, 2, dist, between=between)
+        dense_bytes = sum(wd.seqlens) * wd.Hkv * wd.D * 4
+        out["dense_decode_128k"] = {"ms": msd / 5, "gbs": dense_bytes / (msd / 5 / 1000) / 1e9,
+                                    "speedup_of_sparse_attn": (msd / 5) / a_ms_launch}
+        del wsb
+    del xd, dc
     torch.cuda.empty_cache()
     return out
 
@@ -553,13 +557,18 @@ def one_million(args, dist, pk):
     ms = timed(pf.run, 1, 1, dist)
     flops = selected_flops(pf)
     out["prefill_1m"] = {"ms": ms, "tokens_per_s": dist.world * w.total_rows / (ms / 1000),
-                         "tflops_selected": flops / (ms / 1000) / 1e12}
-    od = torch.empty_like(pf.o)
-    ld = torch.empty_like(pf.lse)
-    T = pf.shape.total_rows
-    msd = timed(lambda: msa.msa_dense_attn_prefill(pf.cfg, pf.shape, x["q"], x["k"], x["v"], 0, T, od, ld), 1, 0, dist)
-    out["dense_prefill_1m"] = {"ms": msd, "tflops": dense_flops(w) / (msd / 1000) / 1e12, "speedup_of_sparse": msd / ms}
-    del x, pf, od, ld
+                         "tflops_selected": flops / (ms / 1000) / 1e12,
+                         "kernel_ms_one_step": family_split(msa, pf)}
+    if not args.no_dense:
+        od = torch.empty_like(pf.o)
+        ld = torch.empty_like(pf.lse)
+        T = pf.shape.total_rows
+        msd = timed(lambda: msa.msa_dense_attn_prefill(pf.cfg, pf.shape, x["q"], x["k"], x["v"], 0, T, od, ld), 1, 0,
+                    dist)
+        out["dense_prefill_1m"] = {"ms": msd, "tflops": dense_flops(w) / (msd / 1000) / 1e12,
+                                   "speedup_of_sparse": msd / ms}
+        del od, ld
+    del x, pf
     torch.cuda.empty_cache()
     wd = WORKLOADS["decode_1m"]
     xd = make_inputs(wd, device="cuda", seed=300 + dist.rank)
@@ -575,11 +584,12 @@ def one_million(args, dist, pk):
                         "attn_ms": a_ms, "selected_bytes": sel, "attn_gbs": sel / (a_ms / 1000) / 1e9,
                         "hbm_frac": sel / (a_ms / 1000) / 1e9 / float(pk["hbm_gbs"]), "graph": True, "l2": L2_NOTE}
     del attn
-    ws = msa.msa_dense_attn_decode(dc.cfg, dc.shape, None, None, None, None, None, None)
-    wsb = torch.empty(ws, dtype=torch.uint8, device="cuda")
-    msd = timed(lambda: msa.msa_dense_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.o, dc.lse, wsb),
-                3, 1, dist, between=between)
-    out["dense_decode_1m"] = {"ms": msd / 3, "speedup_of_sparse_step": (msd / 3) / (ms / 20)}
+    if not args.no_dense:
+        ws = msa.msa_dense_attn_decode(dc.cfg, dc.shape, None, None, None, None, None, None)
+        wsb = torch.empty(ws, dtype=torch.uint8, device="cuda")
+        msd = timed(lambda: msa.msa_dense_attn_decode(dc.cfg, dc.shape, xd["q"], xd["k"], xd["v"], dc.o, dc.lse,
+                                                      wsb), 3, 1, dist, between=between)
+        out["dense_decode_1m"] = {"ms": msd / 3, "speedup_of_sparse_step": (msd / 3) / (ms / 20)}
     return out
 
 

@@ -106,6 +106,7 @@ msa_status_t check_cfg(const msa_config_t *c) {
     if (c->block_size != 64 && c->block_size != 128) return MSA_ERR_UNSUPPORTED;
     if (c->index_dim != 64) return MSA_ERR_UNSUPPORTED;
     if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return MSA_ERR_UNSUPPORTED;
+    if (c->num_kv_heads > 64) return MSA_ERR_UNSUPPORTED;   // block keys stage [5][Hkv][D] fp32 in smem
     if (c->n_topk + 1 + c->use_sink > 256) return MSA_ERR_UNSUPPORTED;
     return MSA_OK;
 }
@@ -305,7 +306,10 @@ msa_status_t msa_index_scores(const msa_config_t *cfg, const msa_shape_t *shape,
     const Prob P = make_prob(cfg, shape, row_begin, row_end, nullptr);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int launched = 0;
-    if (k) {
+    // the newest block of a decode sequence is never scored in its own step, so its key is
+    // computed after (and overlapping) the scoring kernel; every other key comes first
+    const bool newest = kidx_from_block == MSA_KIDX_NEWEST_BLOCK;
+    if (k && !newest) {
         cudaError_t e = launch_block_keys(P, k, wk, k_idx, kidx_from_block, s);
         if (e != cudaSuccess) return MSA_ERR_CUDA;
         ++launched;
@@ -321,8 +325,45 @@ msa_status_t msa_index_scores(const msa_config_t *cfg, const msa_shape_t *shape,
         e = launch_index_scores_prefill(P, tm, q, wq, scores, scores_row_stride, q_idx_out, s);
     } else {
         e = launch_index_scores_decode(P, q, wq, k_idx, scores, scores_row_stride, q_idx_out, s);
+        if (e == cudaSuccess && row_end > row_begin) ++launched;
+        if (e == cudaSuccess && k && newest) {
+            // trailing only when the scoring kernel ran just before (it waited for earlier work)
+            e = launch_block_keys(P, k, wk, k_idx, kidx_from_block, s, row_end > row_begin);
+            ++launched;
+        }
+        return cuda_status(e, launched);
     }
     return cuda_status(e, launched + (row_end > row_begin ? 1 : 0));
+}
+
+msa_status_t msa_index_topk(const msa_config_t *cfg, const msa_shape_t *shape, const void *q, const void *k,
+                            const void *wq, const void *wk, void *k_idx, int64_t kidx_from_block, int64_t row_begin,
+                            int64_t row_end, int32_t *block_idx, void *q_idx_out, int32_t *err_flag, void *stream) {
+    msa_status_t st = check_cfg(cfg);
+    if (st != MSA_OK) return st;
+    if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
+    if (shape->mode != MSA_PREFILL) return MSA_ERR_UNSUPPORTED;
+    if (!q || !wq || !k_idx || !block_idx || (k && !wk)) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(wq, 16) || !aligned(k_idx, 16) || !aligned(block_idx, 4) ||
+        (k && (!aligned(k, 16) || !aligned(wk, 16))) || (q_idx_out && !aligned(q_idx_out, 16)))
+        return MSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_end < row_begin || row_end > shape->total_rows || kidx_from_block < 0)
+        return MSA_ERR_INVALID_ARG;
+    const Prob P = make_prob(cfg, shape, row_begin, row_end, err_flag);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int launched = 0;
+    if (k) {
+        if (launch_block_keys(P, k, wk, k_idx, kidx_from_block, s) != cudaSuccess) return MSA_ERR_CUDA;
+        ++launched;
+    }
+    if (P.total_blocks == 0 || row_end == row_begin) return cuda_status(cudaSuccess, launched);
+    CUtensorMap tm;
+    const uint64_t dims[3] = {64, (uint64_t)P.Hkv, (uint64_t)P.total_blocks};
+    const uint64_t strides[2] = {128, (uint64_t)P.Hkv * 128};
+    const uint32_t box[3] = {64, 1, 128};
+    if (!make_map(&tm, k_idx, 3, dims, strides, box)) return MSA_ERR_CUDA;
+    cudaError_t e = launch_index_topk(P, tm, q, wq, block_idx, q_idx_out, s);
+    return cuda_status(e, launched + 1);
 }
 
 msa_status_t msa_select_topk(const msa_config_t *cfg, const msa_shape_t *shape, const float *scores,

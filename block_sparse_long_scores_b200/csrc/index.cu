@@ -11,6 +11,7 @@
 // tcgen05.mma, fp32 accumulator in TMEM -> registers -> global).  Decode rows (one token per
 // sequence, each against its own cache of block keys) are a batched GEMV on the CUDA cores, bound
 // by the bandwidth of reading the block keys.
+#include "index_query.cuh"
 #include "launch.cuh"
 
 namespace msa {
@@ -19,16 +20,21 @@ namespace msa {
 
 // One CTA per block (prefill: global block number; decode: (b, j), or with from_block < 0 one
 // CTA per sequence b for its newest token's block j = (seqlens[b] - 1) / B); 256 threads.
-// smem: kbar [Hkv][D] fp32, W_k [D][d] bf16.
+// smem: kbar [Hkv][D] fp32, W_k [D][d] bf16, partial sums [4][Hkv][D] fp32.
+// `trailing`: launched right after a kernel that has already waited for all earlier work (the
+// decode scoring kernel), so the inputs are ready on entry; the wait then only comes before exit,
+// which keeps completion ordered along the stream while this kernel overlaps the one before it.
 __global__ void __launch_bounds__(256) block_keys_kernel(Prob P, const __nv_bfloat16 *__restrict__ K,
                                                          const __nv_bfloat16 *__restrict__ Wk,
-                                                         __nv_bfloat16 *__restrict__ kidx, int64_t from_block) {
+                                                         __nv_bfloat16 *__restrict__ kidx, int64_t from_block,
+                                                         int trailing) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *kbar = reinterpret_cast<float *>(smem_raw);
     __nv_bfloat16 *Ws = reinterpret_cast<__nv_bfloat16 *>(smem_raw + sizeof(float) * P.Hkv * P.D);
+    float *part = reinterpret_cast<float *>(smem_raw + sizeof(float) * P.Hkv * P.D + sizeof(__nv_bfloat16) * P.D * P.d);
     const int tid = threadIdx.x;
     const int D = P.D, d = P.d, Hkv = P.Hkv, B = P.B;
-    griddep_wait();     // lengths and cache rows may come from earlier work in the stream
+    if (!trailing) griddep_wait();     // lengths and cache rows may come from earlier work in the stream
     griddep_launch();
 
     int b;
@@ -49,19 +55,27 @@ __global__ void __launch_bounds__(256) block_keys_kernel(Prob P, const __nv_bflo
         len = decode_len(P, b);
     }
     nblk = (len + B - 1) / B;
-    if (j < from_block || j >= nblk || j >= P.max_blocks) return;
+    if (j < from_block || j >= nblk || j >= P.max_blocks) {
+        if (trailing) griddep_wait();
+        return;
+    }
     const int64_t t_first = j * B;
     const int n = (int)lmin(B, len - t_first);
 
     for (int i = tid; i < D * d / 8; i += blockDim.x)
         reinterpret_cast<uint4 *>(Ws)[i] = reinterpret_cast<const uint4 *>(Wk)[i];
 
-    // mean over the block's valid tokens, 8 elements (16 bytes) per thread and token
+    // mean over the block's valid tokens: 16-byte vectors of K, the tokens split into 4 contiguous
+    // quarters whose sums (4 loads in flight per thread) are added in a fixed order
     const int n8 = Hkv * D / 8;
-    for (int v = tid; v < n8; v += blockDim.x) {
+    const int quarter = (n + 3) / 4;
+    for (int w = tid; w < 4 * n8; w += blockDim.x) {
+        const int v = w % n8, qt = w / n8;
         const int g = (v * 8) / D, e = (v * 8) % D;
+        const int t0 = qt * quarter, t1 = min(n, t0 + quarter);
         float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        for (int t = 0; t < n; ++t) {
+#pragma unroll 4
+        for (int t = t0; t < t1; ++t) {
             int64_t off;
             if (P.mode == 0)
                 off = ((int64_t)P.cu_seqlens[b] + t_first + t) * Hkv * D + (int64_t)g * D + e;
@@ -77,8 +91,11 @@ __global__ void __launch_bounds__(256) block_keys_kernel(Prob P, const __nv_bflo
             }
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) kbar[g * D + e + q] = acc[q] / (float)n;
+        for (int q = 0; q < 8; ++q) part[(qt * Hkv + g) * D + e + q] = acc[q];
     }
+    __syncthreads();
+    for (int x = tid; x < Hkv * D; x += blockDim.x)
+        kbar[x] = (((part[x] + part[Hkv * D + x]) + part[2 * Hkv * D + x]) + part[3 * Hkv * D + x]) / (float)n;
     __syncthreads();
 
     // projection by W_k, rounded once to bf16
@@ -93,46 +110,7 @@ __global__ void __launch_bounds__(256) block_keys_kernel(Prob P, const __nv_bflo
             dst = (((int64_t)b * Hkv + g) * P.max_blocks + j) * d + c;
         kidx[dst] = __float2bfloat16_rn(acc);
     }
-}
-
-// --------------------------------------------------------------- index query, one row, fp32
-
-// qhat[c] = sum_e (mean_h Q[row, g*G + h, e]) * W_q[e][c] for c in [0, 64), from smem W_q.
-template <int D>
-__device__ __forceinline__ void index_query_row(const __nv_bfloat16 *__restrict__ qrow, int G,
-                                                const __nv_bfloat16 *Ws, float (&acc)[64]) {
-#pragma unroll
-    for (int c = 0; c < 64; ++c) acc[c] = 0.f;
-    const float invG = 1.0f / (float)G;
-    for (int e0 = 0; e0 < D; e0 += 8) {
-        float qb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        for (int h = 0; h < G; ++h) {
-            uint4 raw = *reinterpret_cast<const uint4 *>(qrow + (int64_t)h * D + e0);
-            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float2 f = __bfloat1622float2(h2[q]);
-                qb[2 * q] += f.x;
-                qb[2 * q + 1] += f.y;
-            }
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float qv = qb[q] * invG;
-            const uint4 *wrow = reinterpret_cast<const uint4 *>(Ws + (e0 + q) * 64);
-#pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-                uint4 raw = wrow[c8];
-                const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    float2 w = __bfloat1622float2(w2[t]);
-                    acc[c8 * 8 + 2 * t] = fmaf(qv, w.x, acc[c8 * 8 + 2 * t]);
-                    acc[c8 * 8 + 2 * t + 1] = fmaf(qv, w.y, acc[c8 * 8 + 2 * t + 1]);
-                }
-            }
-        }
-    }
+    if (trailing) griddep_wait();
 }
 
 // ------------------------------------------------------------------ prefill scores (tcgen05)
@@ -369,18 +347,18 @@ __global__ void __launch_bounds__(256, 4) index_scores_decode_kernel(Prob P, con
 // ------------------------------------------------------------------------------ launchers
 
 cudaError_t launch_block_keys(const Prob &P, const void *K, const void *Wk, void *kidx, int64_t from_block,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool trailing) {
     const int64_t nctas = P.mode == 0 ? P.total_blocks
                                       : (from_block < 0 ? (int64_t)P.batch : (int64_t)P.batch * P.max_blocks);
     if (nctas == 0) return cudaSuccess;
-    const size_t smem = sizeof(float) * P.Hkv * P.D + sizeof(__nv_bfloat16) * P.D * P.d;
+    const size_t smem = sizeof(float) * P.Hkv * P.D * 5 + sizeof(__nv_bfloat16) * P.D * P.d;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(block_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     ProfScope prof("block_keys", st);
     return launch_pdl(block_keys_kernel, dim3((unsigned)nctas), dim3(256), smem, st, P, (const __nv_bfloat16 *)K,
-                      (const __nv_bfloat16 *)Wk, (__nv_bfloat16 *)kidx, from_block);
+                      (const __nv_bfloat16 *)Wk, (__nv_bfloat16 *)kidx, from_block, trailing ? 1 : 0);
 }
 
 size_t index_tc_smem() { return sizeof(IdxSmem) + 1024; }

@@ -38,14 +38,18 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 }
 
 // index.cu
+// trailing: launched right after the decode scoring kernel, overlapping it (see index.cu)
 cudaError_t launch_block_keys(const Prob &P, const void *K, const void *Wk, void *kidx, int64_t from_block,
-                              cudaStream_t st);
+                              cudaStream_t st, bool trailing = false);
 cudaError_t launch_index_scores_prefill(const Prob &P, const CUtensorMap &tm_kidx, const void *Q, const void *Wq,
                                         float *scores, int64_t stride, void *qidx_out, cudaStream_t st);
 cudaError_t launch_index_scores_decode(const Prob &P, const void *Q, const void *Wq, const void *kidx, float *scores,
                                        int64_t stride, void *qidx_out, cudaStream_t st);
 // topk.cu
 cudaError_t launch_select_topk(const Prob &P, const float *scores, int64_t stride, int32_t *out, cudaStream_t st);
+// index_topk.cu
+cudaError_t launch_index_topk(const Prob &P, const CUtensorMap &tm_kidx, const void *Q, const void *Wq, int32_t *out,
+                              void *qidx_out, cudaStream_t st);
 
 // attn_prefill.cu
 struct PrefillWs {

@@ -29,7 +29,7 @@ DERR = {1: "BLOCK_RANGE", 2: "DUPLICATE", 4: "NAN_SCORE", 8: "TIMEOUT", 16: "SHA
 EXPORTED = ("msa_index_scores", "msa_select_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
             "msa_dense_attn_prefill", "msa_dense_attn_decode", "msa_status_string", "msa_version",
             "msa_launch_count", "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
-            "msa_sparse_attn_decode_noalloc", "msa_profile_only")
+            "msa_sparse_attn_decode_noalloc", "msa_profile_only", "msa_index_topk")
 
 
 class MSAError(RuntimeError):
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
         sig = {
             "msa_index_scores": [CP, SP, P, P, P, P, P, I64, I64, I64, P, I64, P, P],
             "msa_select_topk": [CP, SP, P, I64, I64, I64, P, P, P],
+            "msa_index_topk": [CP, SP, P, P, P, P, P, I64, I64, I64, P, P, P, P],
             "msa_sparse_attn_prefill": [CP, SP, P, P, P, P, I64, I64, P, P, P, SZ, P, P],
             "msa_sparse_attn_decode": [CP, SP, P, P, P, P, P, P, P, SZ, P, P],
             "msa_dense_attn_prefill": [CP, SP, P, P, P, I64, I64, P, P, P, P],
@@ -162,6 +163,16 @@ def msa_select_topk(cfg: Config, shape: Shape, scores, scores_row_stride: int, r
     rc = lib().msa_select_topk(ctypes.byref(cfg), ctypes.byref(shape), _ptr(scores), scores_row_stride,
                                row_begin, row_end, _ptr(block_idx), _ptr(err_flag), _stream(stream))
     _check("msa_select_topk", rc)
+
+
+def msa_index_topk(cfg: Config, shape: Shape, q, k, wq, wk, k_idx, kidx_from_block: int, row_begin: int,
+                   row_end: int, block_idx, q_idx_out=None, err_flag=None, stream=None):
+    """Index scores and per-group top-k in one call (prefill): block_idx [rows, Hkv, k_tot] as
+    msa_index_scores + msa_select_topk would give, without a score buffer."""
+    rc = lib().msa_index_topk(ctypes.byref(cfg), ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(wq), _ptr(wk),
+                              _ptr(k_idx), kidx_from_block, row_begin, row_end, _ptr(block_idx), _ptr(q_idx_out),
+                              _ptr(err_flag), _stream(stream))
+    _check("msa_index_topk", rc)
 
 
 def msa_sparse_attn_prefill(cfg: Config, shape: Shape, q, k, v, block_idx, row_begin: int, row_end: int,

@@ -17,9 +17,14 @@ def _ceil4(x: int) -> int:
 
 
 class Prefill:
-    """Packed prefill of workload `w` on inputs `x` (device tensors from workloads.make_inputs)."""
+    """Packed prefill of workload `w` on inputs `x` (device tensors from workloads.make_inputs).
 
-    def __init__(self, w: Workload, x: dict, chunk_rows: int | None = None, with_lse: bool = True):
+    With `fused` (the default) the index branch is one call per row chunk (msa_index_topk: scores
+    and selection without a score buffer); otherwise msa_index_scores writes the chunk's scores and
+    msa_select_topk selects from them."""
+
+    def __init__(self, w: Workload, x: dict, chunk_rows: int | None = None, with_lse: bool = True,
+                 fused: bool = True):
         assert w.mode == "prefill"
         self.w, self.x = w, x
         dev = x["q"].device
@@ -32,13 +37,22 @@ class Prefill:
         self.chunk = T if chunk_rows is None else max(1, min(chunk_rows, T))
         self.given_kidx = "k_idx" in x
         self.k_idx = x["k_idx"] if self.given_kidx else torch.empty(nblk, w.Hkv, w.d, dtype=torch.bfloat16, device=dev)
-        self.scores = torch.empty(self.chunk, w.Hkv, self.stride, dtype=torch.float32, device=dev)
+        self.fused = fused
+        self._scores = None
         self.block_idx = torch.empty(T, w.Hkv, w.k_tot, dtype=torch.int32, device=dev)
         self.o = torch.empty(T, w.Hq, w.D, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(T, w.Hq, dtype=torch.float32, device=dev) if with_lse else None
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         ws = msa.msa_sparse_attn_prefill(self.cfg, self.shape, None, None, None, None, 0, self.chunk, None, None, None)
         self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+
+    @property
+    def scores(self) -> torch.Tensor:
+        """Score buffer of one row chunk (allocated on first use: the fused path needs none)."""
+        if self._scores is None:
+            self._scores = torch.empty(self.chunk, self.w.Hkv, self.stride, dtype=torch.float32,
+                                       device=self.x["q"].device)
+        return self._scores
 
     def chunks(self):
         T = self.shape.total_rows
@@ -54,18 +68,39 @@ class Prefill:
     def select(self, r0: int, r1: int):
         msa.msa_select_topk(self.cfg, self.shape, self.scores, self.stride, r0, r1, self.block_idx[r0:r1], self.err)
 
+    def index_select(self, r0: int, r1: int, compute_keys: bool, block_idx=None, q_idx_out=None):
+        """Fused index branch for rows [r0, r1) into block_idx (default: this pass's own)."""
+        x = self.x
+        k = None if (self.given_kidx or not compute_keys) else x["k"]
+        out = self.block_idx[r0:r1] if block_idx is None else block_idx
+        msa.msa_index_topk(self.cfg, self.shape, x["q"], k, x["wq"], x["wk"], self.k_idx, 0, r0, r1, out,
+                           q_idx_out, self.err)
+
+    def _index_branch(self, r0: int, r1: int, first: bool):
+        if self.fused:
+            self.index_select(r0, r1, compute_keys=first)
+        else:
+            self.index(r0, r1, compute_keys=first)
+            self.select(r0, r1)
+
     def attend(self, r0: int, r1: int):
         x = self.x
         msa.msa_sparse_attn_prefill(self.cfg, self.shape, x["q"], x["k"], x["v"], self.block_idx[r0:r1], r0, r1,
                                     self.o, self.lse, self.workspace, self.err)
 
     def run(self):
-        """One pass of the whole hot path over every row."""
+        """One pass of the whole hot path over every row.  The fused index branch needs no score
+        buffer, so it selects for all rows in one call; attention runs chunk by chunk (its
+        workspace grows with the rows of a call)."""
+        if self.fused:
+            self.index_select(0, self.shape.total_rows, compute_keys=True)
+            for r0, r1 in self.chunks():
+                self.attend(r0, r1)
+            return self.o, self.lse
         first = True
         for r0, r1 in self.chunks():
-            self.index(r0, r1, compute_keys=first)
+            self._index_branch(r0, r1, first)
             first = False
-            self.select(r0, r1)
             self.attend(r0, r1)
         return self.o, self.lse
 
@@ -94,9 +129,8 @@ class Prefill:
         first = True
         for c, (r0, r1) in enumerate(self.chunks()):
             cur.wait_event(ready[c])
-            self.index(r0, r1, compute_keys=first)
+            self._index_branch(r0, r1, first)
             first = False
-            self.select(r0, r1)
             self.attend(r0, r1)
             done = torch.cuda.Event()
             done.record(cur)

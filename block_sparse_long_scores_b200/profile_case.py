@@ -28,6 +28,7 @@ def main(argv=None) -> int:
     ap.add_argument("--batch", type=int, default=0)
     ap.add_argument("--chunk-rows", type=int, default=16384)
     ap.add_argument("--steps", type=int, default=2)
+    ap.add_argument("--unfused", action="store_true", help="prefill: index scores + top-k as two calls")
     a = ap.parse_args(argv)
     w = WORKLOADS[a.workload]
     if w.mode == "decode" and (a.seq_len or a.batch):
@@ -37,7 +38,7 @@ def main(argv=None) -> int:
         w = scaled_down(w, (a.seq_len,))
     x = make_inputs(w, device="cuda")
     if w.mode == "prefill":
-        job = Prefill(w, x, chunk_rows=a.chunk_rows)
+        job = Prefill(w, x, chunk_rows=a.chunk_rows, fused=not a.unfused)
     else:
         job = Decode(w, x)
         job.prepare_keys()

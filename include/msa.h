@@ -20,6 +20,7 @@
  *   msa_select_topk          per-group exp-free top-k, local/sink added         (index branch)
  *   msa_sparse_attn_prefill  exact attention over the selected blocks, packed   (main branch)
  *   msa_sparse_attn_decode   the same for one new token per sequence            (main branch)
+ * and msa_index_topk fuses the first two for prefill (same result, no score buffer).
  * plus the dense causal GQA kernels that serve as the in-run speed-up baseline (msa_dense_*),
  * and small helpers.
  *
@@ -94,7 +95,7 @@ typedef enum {
 
 typedef struct {
     int32_t num_q_heads;    /* Hq                                                             */
-    int32_t num_kv_heads;   /* Hkv; G = Hq / Hkv heads share a KV head (a GQA group)         */
+    int32_t num_kv_heads;   /* Hkv <= 64; G = Hq / Hkv heads share a KV head (a GQA group)   */
     int32_t head_dim;       /* D: 64 or 128                                                   */
     int32_t block_size;     /* B: tokens per KV block, 64 or 128                              */
     int32_t index_dim;      /* d: 64                                                          */
@@ -164,6 +165,26 @@ msa_status_t msa_select_topk(const msa_config_t *cfg, const msa_shape_t *shape,
                              const float *scores, int64_t scores_row_stride,
                              int64_t row_begin, int64_t row_end,
                              int32_t *block_idx, int32_t *err_flag, void *stream);
+
+/*
+ * msa_index_topk -- the index branch in one call, prefill only: msa_index_scores followed by
+ * msa_select_topk without the score buffer.
+ * Source: the digest's two-branch flowchart ("exp-free Top-k": selecting blocks costs next to
+ * nothing, so the raw logits need not be stored) and "深度解析 MiniMax-M3", section "架构核心：MoE
+ * 与 MSA 的深度融合", item 1 (top-k per GQA group).
+ *  Arguments as msa_index_scores (k, wk, k_idx, kidx_from_block, the row range, q_idx_out) and
+ *  msa_select_topk (block_idx, err_flag).  block_idx equals, entry for entry, what those two
+ *  calls produce for the same rows: the scores are computed by the same tensor-core instruction
+ *  sequence, bit for bit, and selected by the same rule (the min(n_topk, |C|) largest, ties to
+ *  the lower block, NaN skipped and flagged, sink / local added, ascending, -1 padded).  The
+ *  scores are recomputed for each 8-bit digit of the selection instead of being stored, so rows
+ *  are not limited by a score buffer.  Decode mode returns MSA_ERR_UNSUPPORTED.
+ */
+msa_status_t msa_index_topk(const msa_config_t *cfg, const msa_shape_t *shape,
+                            const void *q, const void *k, const void *wq, const void *wk,
+                            void *k_idx, int64_t kidx_from_block,
+                            int64_t row_begin, int64_t row_end,
+                            int32_t *block_idx, void *q_idx_out, int32_t *err_flag, void *stream);
 
 /*
  * msa_sparse_attn_prefill -- main branch, packed prefill.

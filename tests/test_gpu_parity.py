@@ -37,10 +37,12 @@ def _prefill_full_check(w, x, chunk_rows=None, rows=None, check_keys=True):
     qidx_gpu = torch.empty(pf.chunk, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV)
     qidx_rows = np.zeros((len(rows), w.Hkv, w.d), np.uint16)
     first = True
+    fused_idx = torch.full_like(pf.block_idx, -2)
     for r0, r1 in pf.chunks():
         pf.index(r0, r1, compute_keys=first, q_idx_out=qidx_gpu)
         first = False
         pf.select(r0, r1)
+        pf.index_select(r0, r1, compute_keys=False, block_idx=fused_idx[r0:r1])
         pf.attend(r0, r1)
         sel = (rows >= r0) & (rows < r1)
         if sel.any():
@@ -48,6 +50,8 @@ def _prefill_full_check(w, x, chunk_rows=None, rows=None, check_keys=True):
             qidx_rows[sel] = _bits(qidx_gpu[torch.as_tensor(rows[sel] - r0, device=DEV)])
     torch.cuda.synchronize()
     assert int(pf.err.item()) == 0, f"device error flag {int(pf.err.item())}"
+    # the fused index branch selects exactly what scores + selection do, on every row
+    assert torch.equal(fused_idx, pf.block_idx), "fused index-topk differs from index scores + top-k"
     # index branch
     if "k_idx" in xc:
         kidx_ref = _bits(xc["k_idx"])
@@ -441,10 +445,12 @@ def _prefill_sampled_check(w, x, rows, chunk_rows):
     qidx_gpu = torch.empty(pf.chunk, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV)
     qidx_rows = np.zeros((len(rows), w.Hkv, w.d), np.uint16)
     first = True
+    fused_idx = torch.full_like(pf.block_idx, -2)
     for r0, r1 in pf.chunks():
         pf.index(r0, r1, compute_keys=first, q_idx_out=qidx_gpu)
         first = False
         pf.select(r0, r1)
+        pf.index_select(r0, r1, compute_keys=False, block_idx=fused_idx[r0:r1])
         pf.attend(r0, r1)
         sel = (rows >= r0) & (rows < r1)
         if sel.any():
@@ -453,6 +459,7 @@ def _prefill_sampled_check(w, x, rows, chunk_rows):
             qidx_rows[sel] = _bits(qidx_gpu[loc])
     torch.cuda.synchronize()
     assert int(pf.err.item()) == 0
+    assert torch.equal(fused_idx, pf.block_idx), "fused index-topk differs from index scores + top-k"
     xc = {"q": _sparse_rows_cpu(x["q"], rows), "k": x["k"].cpu(), "v": x["v"].cpu(), "wq": x["wq"].cpu(),
           "wk": x["wk"].cpu(), "cu_seqlens": x["cu_seqlens"].cpu(), "cu_blocks": x["cu_blocks"].cpu()}
     sh = oracle_shape(w, xc)
