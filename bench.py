@@ -437,17 +437,18 @@ def main():
     dist.close()
 
 
-def family_split(msa, pf) -> dict:
-    """Milliseconds per kernel family of one untimed pass (every launch bracketed by events)."""
+def family_split(msa, job) -> dict:
+    """Milliseconds per kernel family of one untimed eager pass of a prefill or decode step (every
+    launch bracketed by events)."""
     torch.cuda.synchronize()
     msa.profile_reset()
     msa.profile_enable(True)
-    pf.run()
+    job.run()
     torch.cuda.synchronize()
     msa.profile_enable(False)
     fam = {}
     for f in ("block_keys", "index_scores", "select_topk", "index_topk", "prefill_lists", "prefill_attn",
-              "prefill_combine"):
+              "prefill_combine", "decode_attn"):
         t, n = msa.profile_read(f)
         if n:
             fam[f] = round(t, 3)
@@ -527,9 +528,11 @@ def secondary_measurements(args, dist, pf, x, sparse_ms, pk):
     a_ms_launch = timed(attn.replay, 20, 3, dist, between=between) / 20
     sel_bytes = decode_selected_bytes(dc)
     gbs = sel_bytes / (a_ms_launch / 1000) / 1e9
+    between()
     out["decode_128k"] = {"tokens_per_s": dist.world * wd.batch * 20 / (ms / 1000), "ms_per_step": ms / 20,
                           "attn_ms": a_ms_launch, "selected_bytes": sel_bytes, "attn_gbs": gbs,
-                          "hbm_frac": gbs / float(pk["hbm_gbs"]), "graph": True, "l2": L2_NOTE}
+                          "hbm_frac": gbs / float(pk["hbm_gbs"]), "graph": True, "l2": L2_NOTE,
+                          "kernel_ms_one_eager_step": family_split(msa, dc)}
     del attn
     if not args.no_dense:
         ws = msa.msa_dense_attn_decode(dc.cfg, dc.shape, None, None, None, None, None, None)
@@ -580,9 +583,11 @@ def one_million(args, dist, pk):
                                                        dc.o, dc.lse, dc.workspace, dc.err))
     a_ms = timed(attn.replay, 20, 3, dist, between=between) / 20
     sel = decode_selected_bytes(dc)
+    between()
     out["decode_1m"] = {"ms_per_step": ms / 20, "tokens_per_s": dist.world * wd.batch * 20 / (ms / 1000),
                         "attn_ms": a_ms, "selected_bytes": sel, "attn_gbs": sel / (a_ms / 1000) / 1e9,
-                        "hbm_frac": sel / (a_ms / 1000) / 1e9 / float(pk["hbm_gbs"]), "graph": True, "l2": L2_NOTE}
+                        "hbm_frac": sel / (a_ms / 1000) / 1e9 / float(pk["hbm_gbs"]), "graph": True, "l2": L2_NOTE,
+                        "kernel_ms_one_eager_step": family_split(msa, dc)}
     del attn
     if not args.no_dense:
         ws = msa.msa_dense_attn_decode(dc.cfg, dc.shape, None, None, None, None, None, None)

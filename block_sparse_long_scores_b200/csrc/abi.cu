@@ -287,6 +287,9 @@ int32_t msa_version(void) { return 100; }
 
 int64_t msa_launch_count(void) { return g_launches.load(); }
 
+void msa_prefill_set_subchunk_rows(int64_t rows) { prefill_set_subchunk_rows(rows); }
+int64_t msa_prefill_subchunk_rows(void) { return prefill_subchunk_rows(); }
+
 msa_status_t msa_index_scores(const msa_config_t *cfg, const msa_shape_t *shape, const void *q, const void *k,
                               const void *wq, const void *wk, void *k_idx, int64_t kidx_from_block, int64_t row_begin,
                               int64_t row_end, float *scores, int64_t scores_row_stride, void *q_idx_out,
@@ -397,7 +400,7 @@ msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t 
     if (R >= ((int64_t)1 << 23) || R * cfg->num_kv_heads * (cfg->n_topk + 1 + cfg->use_sink) >= ((int64_t)1 << 31))
         return MSA_ERR_UNSUPPORTED;
     const Prob P = make_prob(cfg, shape, row_begin, row_end, err_flag);
-    const size_t need = prefill_ws_layout(P, R, nullptr).total;
+    const size_t need = prefill_ws_bytes(P, R);
     if (!workspace) {
         *workspace_bytes = need;
         return MSA_OK;
@@ -412,7 +415,7 @@ msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t 
     if (!prefill_maps(P, q, k, v, &tq, &tk, &tv)) return MSA_ERR_CUDA;
     cudaError_t e = launch_sparse_prefill(P, tq, tk, tv, q, block_idx, o, lse, workspace, num_sms(),
                                           static_cast<cudaStream_t>(stream));
-    return cuda_status(e, 6);
+    return cuda_status(e, 6 * (int)ceil_div<int64_t>(R, prefill_subchunk_rows()));
 }
 
 msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *shape, const void *q,

@@ -19,6 +19,9 @@
 //   tiles    cut each list into tiles of at most 128/max(G,8) tokens
 //   attn     persistent tcgen05 kernel over the tiles
 //   combine  merge each (row, group)'s partials into O and lse
+#include <algorithm>
+#include <atomic>
+
 #include "launch.cuh"
 
 namespace msa {
@@ -813,12 +816,30 @@ static cudaError_t launch_combine_t(const Prob &P, const PrefillWs &w, void *O, 
         default: return cudaErrorInvalidValue;                                                      \
     }
 
-cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                  const void *q, const int32_t *block_idx, void *O, float *lse, void *ws, int num_sms,
-                                  cudaStream_t st) {
+// ------------------------------------------------------------------------- row sub-chunks
+//
+// A call's rows are processed in sub-chunks of at most prefill_subchunk_rows() rows, each with its
+// own list building, attention and combine, alternating between two workspace halves, so a call
+// over any number of rows needs two sub-chunks' workspace.  (Running a sub-chunk's combine beside
+// the next sub-chunk's attention was tried: the attention kernel, paced by its issue slots and
+// shared-memory traffic, ran about twice as slowly with a combine CTA on each SM.)
+
+static std::atomic<int64_t> g_sub_rows{16384};
+
+void prefill_set_subchunk_rows(int64_t rows) { g_sub_rows.store(rows > 0 ? rows : 16384); }
+int64_t prefill_subchunk_rows() { return g_sub_rows.load(); }
+
+size_t prefill_ws_bytes(const Prob &P, int64_t R) {
+    const int64_t S = prefill_subchunk_rows();
+    if (R <= S) return prefill_ws_layout(P, R, nullptr).total;
+    return 2 * align256(prefill_ws_layout(P, S, nullptr).total);
+}
+
+// Lists, attention and combine of the rows of P, with workspace `w`.
+static cudaError_t prefill_one(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                               const void *q, const int32_t *block_idx, void *O, float *lse, const PrefillWs &w,
+                               int num_sms, cudaStream_t st) {
     const int64_t R = P.row_end - P.row_begin;
-    if (R <= 0) return cudaSuccess;
-    const PrefillWs w = prefill_ws_layout(P, R, ws);
     const int rpt = P.G < 8 ? 8 : P.G;
     const int tpt = 128 / rpt;
     const int64_t L = (int64_t)P.Hkv * P.total_blocks;
@@ -854,6 +875,27 @@ cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CU
     if (P.D == 128) { MSA_DISPATCH_G(P.G, e = launch_combine_t<128, G_>(P, w, O, lse, st)); }
     else { MSA_DISPATCH_G(P.G, e = launch_combine_t<64, G_>(P, w, O, lse, st)); }
     return e;
+}
+
+cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                  const void *q, const int32_t *block_idx, void *O, float *lse, void *ws, int num_sms,
+                                  cudaStream_t st) {
+    const int64_t R = P.row_end - P.row_begin;
+    if (R <= 0) return cudaSuccess;
+    const int64_t S = prefill_subchunk_rows();
+    if (R <= S) return prefill_one(P, tq, tk, tv, q, block_idx, O, lse, prefill_ws_layout(P, R, ws), num_sms, st);
+    const size_t half = align256(prefill_ws_layout(P, S, nullptr).total);
+    const PrefillWs wb[2] = {prefill_ws_layout(P, S, ws), prefill_ws_layout(P, S, static_cast<char *>(ws) + half)};
+    const int64_t n_sub = ceil_div<int64_t>(R, S);
+    for (int64_t c = 0; c < n_sub; ++c) {
+        Prob Pc = P;
+        Pc.row_begin = P.row_begin + c * S;
+        Pc.row_end = std::min<int64_t>(P.row_end, Pc.row_begin + S);
+        cudaError_t e = prefill_one(Pc, tq, tk, tv, q, block_idx + (c * S) * P.Hkv * (int64_t)P.k_tot, O, lse,
+                                    wb[c & 1], num_sms, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace msa

@@ -60,6 +60,9 @@ struct PrefillWs {
     size_t total;
 };
 PrefillWs prefill_ws_layout(const Prob &P, int64_t R, void *base);
+size_t prefill_ws_bytes(const Prob &P, int64_t R);          // workspace of a call over R rows
+void prefill_set_subchunk_rows(int64_t rows);                // rows per internal sub-chunk (<= 0: default)
+int64_t prefill_subchunk_rows();
 cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const void *q, const int32_t *block_idx, void *O, float *lse, void *ws,
                                   int num_sms, cudaStream_t st);

@@ -29,7 +29,8 @@ DERR = {1: "BLOCK_RANGE", 2: "DUPLICATE", 4: "NAN_SCORE", 8: "TIMEOUT", 16: "SHA
 EXPORTED = ("msa_index_scores", "msa_select_topk", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
             "msa_dense_attn_prefill", "msa_dense_attn_decode", "msa_status_string", "msa_version",
             "msa_launch_count", "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
-            "msa_sparse_attn_decode_noalloc", "msa_profile_only", "msa_index_topk")
+            "msa_sparse_attn_decode_noalloc", "msa_profile_only", "msa_index_topk",
+            "msa_prefill_set_subchunk_rows", "msa_prefill_subchunk_rows")
 
 
 class MSAError(RuntimeError):
@@ -90,6 +91,10 @@ def lib() -> ctypes.CDLL:
         L.msa_launch_count.restype = I64
         L.msa_profile_enable.argtypes = [ctypes.c_int]
         L.msa_profile_enable.restype = None
+        L.msa_prefill_set_subchunk_rows.argtypes = [I64]
+        L.msa_prefill_set_subchunk_rows.restype = None
+        L.msa_prefill_subchunk_rows.argtypes = []
+        L.msa_prefill_subchunk_rows.restype = I64
         L.msa_profile_only.argtypes = [ctypes.c_char_p]
         L.msa_profile_only.restype = None
         L.msa_profile_reset.argtypes = []
@@ -224,6 +229,15 @@ def msa_dense_attn_decode(cfg: Config, shape: Shape, q, k_cache, v_cache, o, lse
                                      _ptr(err_flag), _stream(stream))
     _check("msa_dense_attn_decode", rc)
     return nbytes.value
+
+
+def prefill_set_subchunk_rows(rows: int):
+    """Rows per internal prefill sub-chunk (<= 0: the default, 16384)."""
+    lib().msa_prefill_set_subchunk_rows(int(rows))
+
+
+def prefill_subchunk_rows() -> int:
+    return int(lib().msa_prefill_subchunk_rows())
 
 
 def launch_count() -> int:

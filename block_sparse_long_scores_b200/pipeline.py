@@ -43,7 +43,9 @@ class Prefill:
         self.o = torch.empty(T, w.Hq, w.D, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(T, w.Hq, dtype=torch.float32, device=dev) if with_lse else None
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
-        ws = msa.msa_sparse_attn_prefill(self.cfg, self.shape, None, None, None, None, 0, self.chunk, None, None, None)
+        # one attention call may cover every row: the library works in sub-chunks and needs at most
+        # two sub-chunks' workspace (enough for any smaller call as well)
+        ws = msa.msa_sparse_attn_prefill(self.cfg, self.shape, None, None, None, None, 0, T, None, None, None)
         self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
 
     @property
@@ -90,12 +92,12 @@ class Prefill:
 
     def run(self):
         """One pass of the whole hot path over every row.  The fused index branch needs no score
-        buffer, so it selects for all rows in one call; attention runs chunk by chunk (its
-        workspace grows with the rows of a call)."""
+        buffer and the attention call works through its rows in sub-chunks (overlapping each
+        sub-chunk's combine with the next one's attention), so both are one call over all rows."""
         if self.fused:
-            self.index_select(0, self.shape.total_rows, compute_keys=True)
-            for r0, r1 in self.chunks():
-                self.attend(r0, r1)
+            T = self.shape.total_rows
+            self.index_select(0, T, compute_keys=True)
+            self.attend(0, T)
             return self.o, self.lse
         first = True
         for r0, r1 in self.chunks():

@@ -59,8 +59,8 @@
  *            otherwise *workspace_bytes must be at least that size (else MSA_ERR_WORKSPACE).
  *            The workspace must be 256-byte aligned and must not be shared by calls that may
  *            run concurrently.
- * Threads.   Calls are re-entrant and thread-safe; the only process state is a per-device cache
- *            of kernel attributes.
+ * Threads.   Calls are re-entrant and thread-safe; the process state is a per-device cache of
+ *            kernel attributes and the prefill sub-chunk setting.
  */
 #ifndef MSA_H_
 #define MSA_H_
@@ -197,8 +197,9 @@ msa_status_t msa_index_topk(const msa_config_t *cfg, const msa_shape_t *shape,
  *    lse[r, h] = ln sum_t exp(scale * Q[r, h] . K[t, g])                  (nullable)
  *  block_idx rows may be in any order; -1 entries are skipped; out-of-range, future and repeated
  *  entries are skipped and flagged in *err_flag (nullable).
- *  Workspace: two-phase (file header); it grows with (row_end - row_begin), so long prefills are
- *  processed in row chunks.
+ *  Rows are processed in internal sub-chunks of msa_prefill_subchunk_rows() rows (16384 by
+ *  default).  Workspace: two-phase (file header); it grows with (row_end - row_begin) up to one
+ *  sub-chunk and is then two sub-chunks' worth whatever the row count.
  *  Supported (head_dim, block_size): (64, 64), (64, 128), (128, 64); (128, 128) returns
  *  MSA_ERR_UNSUPPORTED (the kernel's rings of query, key/value and probability tiles would not fit
  *  an SM's shared memory).
@@ -273,6 +274,11 @@ msa_status_t msa_dense_attn_decode(const msa_config_t *cfg, const msa_shape_t *s
                                    void *o, float *lse,
                                    void *workspace, size_t *workspace_bytes,
                                    int32_t *err_flag, void *stream);
+
+/* Rows per internal prefill sub-chunk (a process-wide tuning setting; <= 0 restores the default
+ * of 16384).  Query workspace sizes under the same setting as the calls that use them. */
+void msa_prefill_set_subchunk_rows(int64_t rows);
+int64_t msa_prefill_subchunk_rows(void);
 
 /* Helpers. */
 const char *msa_status_string(msa_status_t s);

@@ -71,6 +71,24 @@ def test_prefill_workspace_query_is_host_only_and_grows_with_rows(L):
     assert big >= 16384 * 4 * 66 * 8 * 128 * 2
 
 
+def test_prefill_workspace_stops_growing_past_two_subchunks(L):
+    # past one sub-chunk the call alternates two sub-chunk workspaces, whatever the row count
+    cfg, shape = _cfg(), _prefill_shape()
+    assert L.msa_prefill_subchunk_rows() == 16384
+    _, one = _ws(L, cfg, shape, 0, 16384)
+    _, two = _ws(L, cfg, shape, 0, 16385)
+    _, all_rows = _ws(L, cfg, shape, 0, 131072)
+    assert two == all_rows and one < two <= 2 * one + 256
+    L.msa_prefill_set_subchunk_rows(1000)
+    try:
+        assert L.msa_prefill_subchunk_rows() == 1000
+        _, small = _ws(L, cfg, shape, 0, 131072)
+        assert small < one
+    finally:
+        L.msa_prefill_set_subchunk_rows(0)
+    assert L.msa_prefill_subchunk_rows() == 16384
+
+
 def test_decode_workspace_query(L):
     cfg = _cfg()
     shape = msa.Shape(msa.MSA_DECODE, 32, None, None, 0x10000, 32, 0, 131072, 2048)

@@ -118,6 +118,29 @@ def test_ragged_shape_sharp_logits(gain):
     _prefill_full_check(w, x, chunk_rows=1500)
 
 
+def test_prefill_in_subchunks():
+    # one attention call over 6000 rows in sub-chunks of 1000 rows: two alternating workspace halves
+    w = scaled_down(WORKLOADS["prefill_128k"], (6000,))
+    x = make_inputs(w, device=DEV, seed=33, logit_gain=11.3137)
+    msa.prefill_set_subchunk_rows(1000)
+    try:
+        pf = Prefill(w, x)
+        pf.run()
+        o1 = pf.o.clone()
+        pf.o.zero_()
+        pf.run()                                   # again: the halves are reused, results repeat
+        torch.cuda.synchronize()
+        assert int(pf.err.item()) == 0
+        assert torch.equal(o1, pf.o)
+    finally:
+        msa.prefill_set_subchunk_rows(0)
+    xc = cpu(x)
+    sh = oracle_shape(w, xc)
+    rows = np.arange(w.total_rows)
+    O_ref, L_ref = orc.sparse_attn(sh, xc["q"], xc["k"], xc["v"], pf.block_idx.cpu().numpy(), rows)
+    check_attention(pf.o.float().cpu().numpy(), O_ref, pf.lse.cpu().numpy(), L_ref)
+
+
 def test_ragged_prefill_small_with_ties():
     # ragged workload shape (64/8 heads, D 64, B 128, k 32, discrete index keys -> exact ties)
     w = scaled_down(WORKLOADS["ragged_prefill"], (1, 130, 1000, 64, 2900, 129, 700))
