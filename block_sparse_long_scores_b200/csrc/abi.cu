@@ -287,6 +287,12 @@ int32_t msa_version(void) { return 100; }
 
 int64_t msa_launch_count(void) { return g_launches.load(); }
 
+msa_status_t msa_diag_wait_timeout(int32_t *err_flag, int64_t limit_ns, void *stream) {
+    if (!err_flag || !aligned(err_flag, 4) || limit_ns < 1 || limit_ns > (int64_t)kWaitLimitNs)
+        return MSA_ERR_INVALID_ARG;
+    return cuda_status(launch_wait_timeout_probe(err_flag, (uint64_t)limit_ns, static_cast<cudaStream_t>(stream)), 1);
+}
+
 void msa_prefill_set_subchunk_rows(int64_t rows) { prefill_set_subchunk_rows(rows); }
 int64_t msa_prefill_subchunk_rows(void) { return prefill_subchunk_rows(); }
 

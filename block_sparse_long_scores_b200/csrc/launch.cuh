@@ -75,6 +75,8 @@ size_t decode_stream_ws_bytes(const Prob &P, int num_sms);
 cudaError_t launch_decode_stream(const Prob &P, const CUtensorMap &tk, const CUtensorMap &tv, const void *q,
                                  const int32_t *block_idx, void *O, float *lse, void *ws, int num_sms,
                                  cudaStream_t st);
+// diag.cu
+cudaError_t launch_wait_timeout_probe(int *err, uint64_t limit_ns, cudaStream_t st);
 // attn_dense.cu
 cudaError_t launch_dense_prefill(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                  void *O, float *lse, cudaStream_t st);

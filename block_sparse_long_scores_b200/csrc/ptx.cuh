@@ -77,6 +77,17 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
     return ok != 0;
 }
 
+// Wait for the phase with the given parity to complete within limit_ns of %globaltimer; false if
+// the bound ran out.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    const uint32_t hint = (uint32_t)(limit_ns < 1000000ull ? limit_ns : 1000000ull);
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait_sleep(bar, parity, hint)) {
+        if (globaltimer() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
 // Wait for the phase with the given parity to complete; false if the bound ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     // a few suspending tries before the clock is read at all (reading it costs issue slots)

@@ -30,7 +30,7 @@ EXPORTED = ("msa_index_scores", "msa_select_topk", "msa_sparse_attn_prefill", "m
             "msa_dense_attn_prefill", "msa_dense_attn_decode", "msa_status_string", "msa_version",
             "msa_launch_count", "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
             "msa_sparse_attn_decode_noalloc", "msa_profile_only", "msa_index_topk",
-            "msa_prefill_set_subchunk_rows", "msa_prefill_subchunk_rows")
+            "msa_prefill_set_subchunk_rows", "msa_prefill_subchunk_rows", "msa_diag_wait_timeout")
 
 
 class MSAError(RuntimeError):
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
             "msa_dense_attn_prefill": [CP, SP, P, P, P, I64, I64, P, P, P, P],
             "msa_dense_attn_decode": [CP, SP, P, P, P, P, P, P, SZ, P, P],
             "msa_sparse_attn_decode_noalloc": [CP, SP, P, P, P, P, P, P, P, P],
+            "msa_diag_wait_timeout": [P, I64, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -229,6 +230,11 @@ def msa_dense_attn_decode(cfg: Config, shape: Shape, q, k_cache, v_cache, o, lse
                                      _ptr(err_flag), _stream(stream))
     _check("msa_dense_attn_decode", rc)
     return nbytes.value
+
+
+def diag_wait_timeout(err_flag, limit_ns: int, stream=None):
+    """Launch a wait that nothing completes, bounded by limit_ns; it sets MSA_DERR_TIMEOUT."""
+    _check("msa_diag_wait_timeout", lib().msa_diag_wait_timeout(_ptr(err_flag), int(limit_ns), _stream(stream)))
 
 
 def prefill_set_subchunk_rows(rows: int):

@@ -280,6 +280,15 @@ msa_status_t msa_dense_attn_decode(const msa_config_t *cfg, const msa_shape_t *s
 void msa_prefill_set_subchunk_rows(int64_t rows);
 int64_t msa_prefill_subchunk_rows(void);
 
+/*
+ * Diagnostic of the failure handling: launches one thread that waits on a shared-memory barrier
+ * nothing arrives on, bounded (by limit_ns of %globaltimer, 1 ns .. 1 s) exactly like every wait
+ * inside the library's kernels.  When the bound runs out it OR-s MSA_DERR_TIMEOUT into *err_flag
+ * (device int32) and returns, leaving the context usable; this is the path any kernel of this
+ * library takes if one of its internal waits never completes.  No counterpart on the pages.
+ */
+msa_status_t msa_diag_wait_timeout(int32_t *err_flag, int64_t limit_ns, void *stream);
+
 /* Helpers. */
 const char *msa_status_string(msa_status_t s);
 int32_t msa_version(void);            /* major * 10000 + minor * 100 + patch */

@@ -104,3 +104,37 @@ def sample_rows(w, n: int, seed: int = 0):
     extra = rng.integers(0, cu[-1], size=max(0, n - len(rows)))
     rows.update(int(r) for r in extra)
     return np.array(sorted(rows), dtype=np.int64)
+
+
+class Guards:
+    """Guard bands after device buffers: a guarded tensor is a view of a larger allocation whose
+    tail holds a byte pattern; check() asserts that no call wrote past the tensor (or past the
+    workspace size the library reported)."""
+
+    PATTERN = 0xA5
+
+    def __init__(self, tail_bytes: int = 4096):
+        self.tail = tail_bytes
+        self.items = []
+
+    def wrap(self, t: torch.Tensor, name: str = "") -> torch.Tensor:
+        nb = t.numel() * t.element_size()
+        raw = torch.empty(nb + self.tail, dtype=torch.uint8, device=t.device)
+        raw[nb:] = self.PATTERN
+        if nb:
+            raw[:nb].copy_(t.contiguous().view(-1).view(torch.uint8))
+        self.items.append((name, raw, nb))
+        return raw[:nb].view(t.dtype).view(t.shape)
+
+    def guard(self, obj, *names: str):
+        """Replace the listed tensor attributes of obj with guarded copies."""
+        for n in names:
+            t = getattr(obj, n)
+            if t is not None:
+                setattr(obj, n, self.wrap(t, n))
+
+    def check(self):
+        torch.cuda.synchronize()
+        for name, raw, nb in self.items:
+            bad = int((raw[nb:] != self.PATTERN).sum().item())
+            assert bad == 0, f"{bad} guard bytes after '{name}' were overwritten"

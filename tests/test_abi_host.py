@@ -165,6 +165,14 @@ def test_newest_block_key_mode_is_decode_only(L):
     assert rc == 1
 
 
+def test_wait_timeout_diagnostic_checks_its_arguments(L):
+    fake = ctypes.c_void_p(0x100000)
+    assert L.msa_diag_wait_timeout(None, 1000, None) == 1              # no flag to report into
+    assert L.msa_diag_wait_timeout(ctypes.c_void_p(0x100002), 1000, None) == 1   # misaligned
+    assert L.msa_diag_wait_timeout(fake, 0, None) == 1                 # no bound
+    assert L.msa_diag_wait_timeout(fake, 2_000_000_000, None) == 1     # beyond the kernels' 1 s bound
+
+
 def test_select_topk_rejects_misaligned_scores_and_bad_stride(L):
     # long score rows are copied 16 bytes at a time: the base must be 16-byte aligned and the row
     # stride a multiple of 4 floats (at least max_blocks), as for msa_index_scores

@@ -13,8 +13,8 @@ from block_sparse_long_scores_b200 import msa
 from block_sparse_long_scores_b200.pipeline import Decode, Prefill
 from block_sparse_long_scores_b200.workloads import WORKLOADS, make_inputs, scaled_down
 from oracle import oracle as orc
-from tests.parity_helpers import (check_attention, check_bf16_near, check_scores, cpu, oracle_shape, row_geometry,
-                                  sample_rows)
+from tests.parity_helpers import (Guards, check_attention, check_bf16_near, check_scores, cpu, oracle_shape,
+                                  row_geometry, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -26,8 +26,12 @@ def _bits(t):
 
 
 def _prefill_full_check(w, x, chunk_rows=None, rows=None, check_keys=True):
-    """Run the prefill path on the GPU and compare each step with the oracle on `rows`."""
+    """Run the prefill path on the GPU and compare each step with the oracle on `rows`; every
+    output, the score buffer and the workspace carry guard bands that must stay untouched."""
     pf = Prefill(w, x, chunk_rows=chunk_rows)
+    guards = Guards()
+    pf.scores  # allocate the score buffer before guarding it
+    guards.guard(pf, "o", "lse", "block_idx", "workspace", "_scores", "k_idx")
     T = pf.shape.total_rows
     rows = np.arange(T) if rows is None else rows
     xc = cpu(x)
@@ -73,6 +77,7 @@ def _prefill_full_check(w, x, chunk_rows=None, rows=None, check_keys=True):
     O_ref, L_ref = orc.sparse_attn(sh, xc["q"], xc["k"], xc["v"], sel_gpu, rows)
     O_gpu = pf.o.float().cpu().numpy()[rows]
     L_gpu = pf.lse.cpu().numpy()[rows]
+    guards.check()
     return check_attention(O_gpu, O_ref, L_gpu, L_ref)
 
 
@@ -238,9 +243,12 @@ def test_block_order_does_not_matter():
 
 def _decode_check(w, x):
     dc = Decode(w, x)
-    qidx = torch.empty(w.batch, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV)
+    guards = Guards()
+    guards.guard(dc, "o", "lse", "block_idx", "workspace", "scores", "k_idx")
+    qidx = guards.wrap(torch.empty(w.batch, w.Hkv, w.d, dtype=torch.bfloat16, device=DEV), "q_idx")
     dc.run(q_idx_out=qidx)
     torch.cuda.synchronize()
+    guards.check()
     return _decode_compare(w, x, dc, qidx)
 
 
@@ -357,6 +365,21 @@ def test_decode_graph_appends_tokens_across_block_boundaries():
         lens = lens0 + t
         assert np.array_equal(x["seqlens"].cpu().numpy(), lens)
         _decode_compare(w.with_(seqlens=tuple(int(v) for v in lens)), x, dc, qidx)
+
+
+def test_wait_timeout_is_reported_and_the_context_stays_usable():
+    # a bounded wait that nothing completes (the path every kernel's internal waits take on a hang):
+    # MSA_DERR_TIMEOUT comes back after the short limit, and the GPU keeps working afterwards
+    import time
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    t0 = time.perf_counter()
+    msa.diag_wait_timeout(err, 2_000_000)          # 2 ms
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 5.0
+    assert int(err.item()) & 8
+    w = scaled_down(WORKLOADS["decode_128k"], (70, 1000))
+    x = make_inputs(w, device=DEV, seed=34)
+    _decode_check(w, x)
 
 
 def test_decode_lengths_beyond_the_cache_are_clamped_and_flagged():
