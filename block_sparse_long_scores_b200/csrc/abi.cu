@@ -424,6 +424,38 @@ msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t 
     return cuda_status(e, 6 * (int)ceil_div<int64_t>(R, prefill_subchunk_rows()));
 }
 
+msa_status_t msa_sparse_attn_prefill_bwd(const msa_config_t *cfg, const msa_shape_t *shape, const void *q,
+                                         const void *k, const void *v, const void *o, const float *lse,
+                                         const void *d_o, const int32_t *block_idx, int64_t row_begin,
+                                         int64_t row_end, float *dq, float *dk, float *dv, void *workspace,
+                                         size_t *workspace_bytes, int32_t *err_flag, void *stream) {
+    msa_status_t st = check_cfg(cfg);
+    if (st != MSA_OK) return st;
+    if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
+    if (shape->mode != MSA_PREFILL || !workspace_bytes) return MSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_end < row_begin || row_end > shape->total_rows) return MSA_ERR_INVALID_ARG;
+    if (cfg->head_dim == 128 && cfg->block_size == 128) return MSA_ERR_UNSUPPORTED;
+    const int64_t R = row_end - row_begin;
+    if (R >= ((int64_t)1 << 23) || R * cfg->num_kv_heads * (cfg->n_topk + 1 + cfg->use_sink) >= ((int64_t)1 << 31))
+        return MSA_ERR_UNSUPPORTED;
+    const Prob P = make_prob(cfg, shape, row_begin, row_end, err_flag);
+    const size_t need = prefill_bwd_ws_bytes(P, R);
+    if (!workspace) {
+        *workspace_bytes = need;
+        return MSA_OK;
+    }
+    if (*workspace_bytes < need) return MSA_ERR_WORKSPACE;
+    if (!q || !k || !v || !o || !lse || !d_o || !block_idx || !dq || !dk || !dv) return MSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(d_o, 16) ||
+        !aligned(lse, 4) || !aligned(block_idx, 4) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+        !aligned(workspace, 256))
+        return MSA_ERR_INVALID_ARG;
+    if (R == 0) return MSA_OK;
+    cudaError_t e = launch_sparse_prefill_bwd(P, q, k, v, o, lse, d_o, block_idx, dq, dk, dv, workspace, num_sms(),
+                                              static_cast<cudaStream_t>(stream));
+    return cuda_status(e, 6 * (int)ceil_div<int64_t>(R, prefill_subchunk_rows()));
+}
+
 msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *shape, const void *q,
                                     const void *k_cache, const void *v_cache, const int32_t *block_idx, void *o,
                                     float *lse, void *workspace, size_t *workspace_bytes, int32_t *err_flag,

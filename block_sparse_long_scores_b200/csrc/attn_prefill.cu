@@ -751,8 +751,9 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(Prob P, const int3
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Workspace carve-up for R rows.  `base` may be null (size query).
-PrefillWs prefill_ws_layout(const Prob &P, int64_t R, void *base) {
+// Workspace carve-up for R rows.  `base` may be null (size query); without `partials` only the
+// list arrays are laid out (the backward pass needs no split partials).
+PrefillWs prefill_ws_layout(const Prob &P, int64_t R, void *base, bool partials) {
     const int rpt = P.G < 8 ? 8 : P.G;
     const int tpt = 128 / rpt;
     const int64_t L = (int64_t)P.Hkv * P.total_blocks;
@@ -772,8 +773,10 @@ PrefillWs prefill_ws_layout(const Prob &P, int64_t R, void *base) {
     w.tile_off = (int32_t *)take(sizeof(int32_t) * (L + 1));
     w.entries = (int32_t *)take(sizeof(int32_t) * E);
     w.tiles = (int4 *)take(sizeof(int4) * max_tiles);
-    w.part_o = (__nv_bfloat16 *)take(sizeof(__nv_bfloat16) * E * P.G * P.D);
-    w.part_ml = (float2 *)take(sizeof(float2) * E * P.G);
+    if (partials) {
+        w.part_o = (__nv_bfloat16 *)take(sizeof(__nv_bfloat16) * E * P.G * P.D);
+        w.part_ml = (float2 *)take(sizeof(float2) * E * P.G);
+    }
     w.total = off;
     return w;
 }
@@ -831,20 +834,18 @@ int64_t prefill_subchunk_rows() { return g_sub_rows.load(); }
 
 size_t prefill_ws_bytes(const Prob &P, int64_t R) {
     const int64_t S = prefill_subchunk_rows();
-    if (R <= S) return prefill_ws_layout(P, R, nullptr).total;
-    return 2 * align256(prefill_ws_layout(P, S, nullptr).total);
+    if (R <= S) return prefill_ws_layout(P, R, nullptr, true).total;
+    return 2 * align256(prefill_ws_layout(P, S, nullptr, true).total);
 }
 
-// Lists, attention and combine of the rows of P, with workspace `w`.
-static cudaError_t prefill_one(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                               const void *q, const int32_t *block_idx, void *O, float *lse, const PrefillWs &w,
-                               int num_sms, cudaStream_t st) {
+// Validate the block lists of the rows of P and file every (row, group, block) triple under its
+// (group, block) list: sanitised lists, counts, offsets, entries and tile descriptors in `w`.
+cudaError_t build_prefill_lists(const Prob &P, const int32_t *block_idx, const PrefillWs &w, cudaStream_t st) {
     const int64_t R = P.row_end - P.row_begin;
     const int rpt = P.G < 8 ? 8 : P.G;
     const int tpt = 128 / rpt;
     const int64_t L = (int64_t)P.Hkv * P.total_blocks;
     cudaError_t e;
-    {
     ProfScope prof("prefill_lists", st);
     if ((e = cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * L, st)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(w.cursor, 0, sizeof(int32_t) * L, st)) != cudaSuccess) return e;
@@ -861,7 +862,16 @@ static cudaError_t prefill_one(const Prob &P, const CUtensorMap &tq, const CUten
     prefill_tiles_kernel<<<(unsigned)ceil_div<int64_t>(L, 256), 256, 0, st>>>(L, tpt, w.counts, w.list_off,
                                                                              w.tile_off, w.tiles);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
+    return cudaSuccess;
+}
+
+// Lists, attention and combine of the rows of P, with workspace `w`.
+static cudaError_t prefill_one(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                               const void *q, const int32_t *block_idx, void *O, float *lse, const PrefillWs &w,
+                               int num_sms, cudaStream_t st) {
+    const int64_t L = (int64_t)P.Hkv * P.total_blocks;
+    cudaError_t e = build_prefill_lists(P, block_idx, w, st);
+    if (e != cudaSuccess) return e;
     PrefillBufs W{static_cast<const __nv_bfloat16 *>(q), w.entries, w.tiles, w.tile_off + L, w.part_o, w.part_ml};
     {
     ProfScope prof("prefill_attn", st);
@@ -883,9 +893,9 @@ cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CU
     const int64_t R = P.row_end - P.row_begin;
     if (R <= 0) return cudaSuccess;
     const int64_t S = prefill_subchunk_rows();
-    if (R <= S) return prefill_one(P, tq, tk, tv, q, block_idx, O, lse, prefill_ws_layout(P, R, ws), num_sms, st);
-    const size_t half = align256(prefill_ws_layout(P, S, nullptr).total);
-    const PrefillWs wb[2] = {prefill_ws_layout(P, S, ws), prefill_ws_layout(P, S, static_cast<char *>(ws) + half)};
+    if (R <= S) return prefill_one(P, tq, tk, tv, q, block_idx, O, lse, prefill_ws_layout(P, R, ws, true), num_sms, st);
+    const size_t half = align256(prefill_ws_layout(P, S, nullptr, true).total);
+    const PrefillWs wb[2] = {prefill_ws_layout(P, S, ws, true), prefill_ws_layout(P, S, static_cast<char *>(ws) + half, true)};
     const int64_t n_sub = ceil_div<int64_t>(R, S);
     for (int64_t c = 0; c < n_sub; ++c) {
         Prob Pc = P;

@@ -59,13 +59,19 @@ struct PrefillWs {
     float2 *part_ml;
     size_t total;
 };
-PrefillWs prefill_ws_layout(const Prob &P, int64_t R, void *base);
+PrefillWs prefill_ws_layout(const Prob &P, int64_t R, void *base, bool partials);
+cudaError_t build_prefill_lists(const Prob &P, const int32_t *block_idx, const PrefillWs &w, cudaStream_t st);
 size_t prefill_ws_bytes(const Prob &P, int64_t R);          // workspace of a call over R rows
 void prefill_set_subchunk_rows(int64_t rows);                // rows per internal sub-chunk (<= 0: default)
 int64_t prefill_subchunk_rows();
 cudaError_t launch_sparse_prefill(const Prob &P, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const void *q, const int32_t *block_idx, void *O, float *lse, void *ws,
                                   int num_sms, cudaStream_t st);
+// attn_bwd.cu
+size_t prefill_bwd_ws_bytes(const Prob &P, int64_t R);
+cudaError_t launch_sparse_prefill_bwd(const Prob &P, const void *q, const void *k, const void *v, const void *o,
+                                      const float *lse, const void *dout, const int32_t *block_idx, float *dq,
+                                      float *dk, float *dv, void *ws, int num_sms, cudaStream_t st);
 // attn_decode.cu
 size_t decode_ws_bytes(const Prob &P, int nct);
 void decode_geometry(const Prob &P, bool dense, int &nct, int &rounds);

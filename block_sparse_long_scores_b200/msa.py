@@ -30,7 +30,8 @@ EXPORTED = ("msa_index_scores", "msa_select_topk", "msa_sparse_attn_prefill", "m
             "msa_dense_attn_prefill", "msa_dense_attn_decode", "msa_status_string", "msa_version",
             "msa_launch_count", "msa_profile_enable", "msa_profile_reset", "msa_profile_read",
             "msa_sparse_attn_decode_noalloc", "msa_profile_only", "msa_index_topk",
-            "msa_prefill_set_subchunk_rows", "msa_prefill_subchunk_rows", "msa_diag_wait_timeout")
+            "msa_prefill_set_subchunk_rows", "msa_prefill_subchunk_rows", "msa_diag_wait_timeout",
+            "msa_sparse_attn_prefill_bwd")
 
 
 class MSAError(RuntimeError):
@@ -77,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "msa_index_topk": [CP, SP, P, P, P, P, P, I64, I64, I64, P, P, P, P],
             "msa_sparse_attn_prefill": [CP, SP, P, P, P, P, I64, I64, P, P, P, SZ, P, P],
             "msa_sparse_attn_decode": [CP, SP, P, P, P, P, P, P, P, SZ, P, P],
+            "msa_sparse_attn_prefill_bwd": [CP, SP, P, P, P, P, P, P, P, I64, I64, P, P, P, P, SZ, P, P],
             "msa_dense_attn_prefill": [CP, SP, P, P, P, I64, I64, P, P, P, P],
             "msa_dense_attn_decode": [CP, SP, P, P, P, P, P, P, SZ, P, P],
             "msa_sparse_attn_decode_noalloc": [CP, SP, P, P, P, P, P, P, P, P],
@@ -190,6 +192,19 @@ def msa_sparse_attn_prefill(cfg: Config, shape: Shape, q, k, v, block_idx, row_b
                                        _ptr(block_idx), row_begin, row_end, _ptr(o), _ptr(lse),
                                        _ptr(workspace), ctypes.byref(nbytes), _ptr(err_flag), _stream(stream))
     _check("msa_sparse_attn_prefill", rc)
+    return nbytes.value
+
+
+def msa_sparse_attn_prefill_bwd(cfg: Config, shape: Shape, q, k, v, o, lse, d_o, block_idx, row_begin: int,
+                                row_end: int, dq, dk, dv, workspace, err_flag=None, stream=None) -> int:
+    """Gradients of the prefill attention for rows [row_begin, row_end), accumulated into the fp32
+    dq [T, Hq, D], dk and dv [T, Hkv, D].  With workspace=None returns the workspace size."""
+    nbytes = ctypes.c_size_t(0 if workspace is None else workspace.numel() * workspace.element_size())
+    rc = lib().msa_sparse_attn_prefill_bwd(ctypes.byref(cfg), ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(o), _ptr(lse), _ptr(d_o), _ptr(block_idx), row_begin, row_end,
+                                           _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ctypes.byref(nbytes),
+                                           _ptr(err_flag), _stream(stream))
+    _check("msa_sparse_attn_prefill_bwd", rc)
     return nbytes.value
 
 

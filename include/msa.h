@@ -213,6 +213,33 @@ msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t 
                                      int32_t *err_flag, void *stream);
 
 /*
+ * msa_sparse_attn_prefill_bwd -- backward of the main branch for packed prefill: gradients of the
+ * attention of msa_sparse_attn_prefill with respect to Q, K and V, the selection held fixed.
+ * Source: the pages report that the model is trained end to end (devpress.csdn.net page, section
+ * "M3的技术局限与改进方向"); what is differentiated is softmax(QK^T/sqrt(d_k))V of the
+ * chenxutan.com page, section 2.1, over the selected blocks.
+ *  For every row r in [row_begin, row_end), head h (kv head g = h / G) and visible key t of its
+ *  selected blocks, with p_t = exp(scale Q[r,h].K[t,g] - lse[r,h]) and D = d_o[r,h] . o[r,h]:
+ *    dv[t, g] += p_t d_o[r, h]
+ *    dq[r, h] += scale dS_t K[t, g],   dk[t, g] += scale dS_t Q[r, h],   dS_t = p_t (d_o[r,h] . V[t,g] - D)
+ *  o and lse are the forward's outputs for these rows ([T, Hq, D] bf16, [T, Hq] fp32); d_o is the
+ *  upstream gradient [T, Hq, D] bf16; block_idx [rows, Hkv, k_tot] as for the forward (validated,
+ *  skipped and flagged the same way).  dq [T, Hq, D], dk and dv [T, Hkv, D] are fp32 and are
+ *  ACCUMULATED into (+=): zero them before the first call; dq receives only the call's rows, dk and
+ *  dv the contributions of the call's rows to every key, so a prefill may be processed in row
+ *  ranges.  Additions from different blocks arrive in no fixed order, so results may differ in the
+ *  last bits between runs.  Workspace: two-phase, one sub-chunk's lists and per-row dot products.
+ *  Supported (head_dim, block_size) as for msa_sparse_attn_prefill.
+ */
+msa_status_t msa_sparse_attn_prefill_bwd(const msa_config_t *cfg, const msa_shape_t *shape,
+                                         const void *q, const void *k, const void *v,
+                                         const void *o, const float *lse, const void *d_o,
+                                         const int32_t *block_idx, int64_t row_begin, int64_t row_end,
+                                         float *dq, float *dk, float *dv,
+                                         void *workspace, size_t *workspace_bytes,
+                                         int32_t *err_flag, void *stream);
+
+/*
  * msa_sparse_attn_decode -- main branch, one new token per sequence against a KV cache.
  * Source: as msa_sparse_attn_prefill; the digest reports decode as the second measured case.
  *  For every sequence b and query head h: the same formula with the token at position

@@ -463,3 +463,97 @@ int orc_dense_attn(const orc_shape *s, const uint16_t *Q, const uint16_t *K, con
     }
     return err;
 }
+
+/*
+ * Backward of the main branch (prefill): the gradients of the attention of orc_sparse_attn with
+ * respect to Q, K and V for an upstream gradient dO, the selection held fixed.  The pages say the
+ * model is trained end to end (devpress.csdn.net page, section "M3的技术局限与改进方向"), which
+ * needs these; what is differentiated is softmax(Q K^T / sqrt(d_k)) V of the chenxutan.com page,
+ * section 2.1, restricted to the selected blocks.  For every row r, head h (group g) and visible
+ * key t of the selected set, with p_t the softmax weight, O the output and D = dO . O:
+ *   dV[t, g] += p_t dO[r, h]
+ *   dS_t      = p_t (dO[r, h] . V[t, g] - D)
+ *   dQ[r, h] += scale dS_t K[t, g]
+ *   dK[t, g] += scale dS_t Q[r, h]
+ * All rows of the prefill are taken (dK and dV gather contributions from every row); the forward
+ * quantities are recomputed here in double.  dQ [T, Hq, D]; dK, dV [T, Hkv, D]; dO is bf16.
+ */
+int orc_sparse_attn_bwd(const orc_shape *s, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                        const uint16_t *dO, const int32_t *block_idx, int k_tot, double scale,
+                        double *dQ, double *dK, double *dV) {
+    if (!s || s->mode != 0 || !Q || !K || !V || !dO || !block_idx || !dQ || !dK || !dV || s->D > 512)
+        return ORC_ERR_ARG;
+    const int D = s->D, G = s->Hq / s->Hkv, B = s->B;
+    const int64_t T = s->T;
+    memset(dQ, 0, sizeof(double) * (size_t)(T * s->Hq * D));
+    memset(dK, 0, sizeof(double) * (size_t)(T * s->Hkv * D));
+    memset(dV, 0, sizeof(double) * (size_t)(T * s->Hkv * D));
+    int err = ORC_OK;
+    /* one KV head per thread: dK and dV of head g only receive contributions of group g */
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int g = 0; g < s->Hkv; ++g) {
+        int64_t cap = 1 << 16;
+        double *z = (double *)malloc(sizeof(double) * (size_t)cap);
+        int64_t *tk = (int64_t *)malloc(sizeof(int64_t) * (size_t)cap);
+        double *o = (double *)malloc(sizeof(double) * (size_t)D);
+        if (!z || !tk || !o) { err = ORC_ERR_MEM; free(z); free(tk); free(o); continue; }
+        for (int64_t r = 0; r < T; ++r) {
+            int b; int64_t pos;
+            if (row_info(s, r, &b, &pos)) { err = ORC_ERR_ARG; break; }
+            const int64_t len = seq_len(s, b);
+            const int64_t s0 = (int64_t)s->cu_seqlens[b];
+            const int32_t *sel = block_idx + (r * s->Hkv + g) * (int64_t)k_tot;
+            int64_t n = 0;
+            for (int a = 0; a < k_tot; ++a) {
+                int32_t j = sel[a];
+                if (j < 0) continue;
+                int dup = 0;
+                for (int c = 0; c < a; ++c) dup |= (sel[c] == j);
+                if (dup) continue;
+                for (int64_t t = (int64_t)j * B; t < (int64_t)(j + 1) * B && t < len && t <= pos; ++t) {
+                    if (n == cap) { err = ORC_ERR_MEM; break; }
+                    tk[n++] = t;
+                }
+            }
+            if (n == 0) continue;
+            for (int h = g * G; h < (g + 1) * G; ++h) {
+                const int64_t qo = q_off(s, r, h);
+                const uint16_t *dOr = dO + qo;
+                /* forward: weights p = softmax(z), output o */
+                double m = -INFINITY;
+                for (int64_t a = 0; a < n; ++a) {
+                    double acc = 0.0;
+                    for (int e = 0; e < D; ++e) acc += bf16_to_double(Q[qo + e]) * kv_at(s, K, b, tk[a], g, e);
+                    z[a] = scale * acc;
+                    if (z[a] > m) m = z[a];
+                }
+                double den = 0.0;
+                for (int64_t a = 0; a < n; ++a) den += exp(z[a] - m);
+                for (int e = 0; e < D; ++e) o[e] = 0.0;
+                for (int64_t a = 0; a < n; ++a) {
+                    z[a] = exp(z[a] - m) / den;   /* z now holds p */
+                    for (int e = 0; e < D; ++e) o[e] += z[a] * kv_at(s, V, b, tk[a], g, e);
+                }
+                double Dd = 0.0;
+                for (int e = 0; e < D; ++e) Dd += bf16_to_double(dOr[e]) * o[e];
+                /* backward */
+                double *dQr = dQ + (r * s->Hq + h) * (int64_t)D;
+                for (int64_t a = 0; a < n; ++a) {
+                    const int64_t kvrow = ((s0 + tk[a]) * s->Hkv + g) * (int64_t)D;
+                    double dp = 0.0;
+                    for (int e = 0; e < D; ++e) dp += bf16_to_double(dOr[e]) * kv_at(s, V, b, tk[a], g, e);
+                    const double ds = z[a] * (dp - Dd);
+                    for (int e = 0; e < D; ++e) {
+                        dV[kvrow + e] += z[a] * bf16_to_double(dOr[e]);
+                        dQr[e] += scale * ds * kv_at(s, K, b, tk[a], g, e);
+                        dK[kvrow + e] += scale * ds * bf16_to_double(Q[qo + e]);
+                    }
+                }
+            }
+        }
+        free(z);
+        free(tk);
+        free(o);
+    }
+    return err;
+}

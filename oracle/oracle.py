@@ -239,3 +239,19 @@ def dense_attn(shape: Shape, Q, K, V, rows, scale: float | None = None):
     _check(_L().orc_dense_attn(ctypes.byref(s), _p(Qb), _p(Kb), _p(Vb), _p(rows), ctypes.c_int64(len(rows)),
                                ctypes.c_double(sc), _p(O), _p(LSE)), "dense_attn")
     return O, LSE
+
+
+def sparse_attn_bwd(shape: Shape, Q, K, V, dO, block_idx: np.ndarray, scale: float | None = None):
+    """Gradients of the selected-block attention for upstream dO (prefill, all rows):
+    dQ [T, Hq, D], dK [T, Hkv, D], dV [T, Hkv, D] (fp64)."""
+    s = shape.c()
+    Qb, Kb, Vb, dOb = _bits(Q), _bits(K), _bits(V), _bits(dO)
+    bi = np.ascontiguousarray(block_idx, dtype=np.int32)
+    k_tot = bi.shape[-1]
+    dQ = np.empty((shape.T, shape.Hq, shape.D), np.float64)
+    dK = np.empty((shape.T, shape.Hkv, shape.D), np.float64)
+    dV = np.empty((shape.T, shape.Hkv, shape.D), np.float64)
+    sc = default_scale(shape.D) if scale is None else scale
+    _check(_L().orc_sparse_attn_bwd(ctypes.byref(s), _p(Qb), _p(Kb), _p(Vb), _p(dOb), _p(bi), ctypes.c_int(k_tot),
+                                    ctypes.c_double(sc), _p(dQ), _p(dK), _p(dV)), "sparse_attn_bwd")
+    return dQ, dK, dV
