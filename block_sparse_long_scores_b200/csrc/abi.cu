@@ -480,7 +480,7 @@ msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *
     if (!decode_maps(P, q, k_cache, v_cache, &tq, &tk, &tv)) return MSA_ERR_CUDA;
     cudaError_t e = launch_decode_stream(P, tk, tv, q, block_idx, o, lse, workspace, num_sms(),
                                          static_cast<cudaStream_t>(stream));
-    return cuda_status(e, 1);
+    return cuda_status(e, 2);
 }
 
 msa_status_t msa_dense_attn_prefill(const msa_config_t *cfg, const msa_shape_t *shape, const void *q, const void *k,
@@ -544,10 +544,10 @@ msa_status_t msa_sparse_attn_decode_noalloc(const msa_config_t *cfg, const msa_s
     if (!scratch) return MSA_ERR_CUDA;
     CUtensorMap tq, tk, tv;
     if (!decode_maps(P, q, k_cache, v_cache, &tq, &tk, &tv)) return MSA_ERR_CUDA;
-    // the scratch needs no clearing: its merge counters are tagged with a per-call generation
+    // the scratch needs no clearing: every partial is written before the merge kernel reads it
     cudaError_t e = launch_decode_stream(P, tk, tv, q, block_idx, o, lse, scratch, num_sms(),
                                          static_cast<cudaStream_t>(stream));
-    return cuda_status(e, 1);
+    return cuda_status(e, 2);
 }
 
 }  // extern "C"

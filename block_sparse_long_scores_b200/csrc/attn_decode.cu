@@ -17,6 +17,7 @@
 // the sparse decode) streams the whole batch's selected blocks through a persistent grid and
 // merges with the same rule.
 #include <algorithm>
+#include <cstddef>
 #include <atomic>
 
 #include "launch.cuh"
@@ -366,7 +367,7 @@ cudaError_t launch_decode(const Prob &P, const CUtensorMap &tq, const CUtensorMa
 // chain of dependent tensor-core and softmax steps per block is a quarter of a whole block's.  Each
 // warp keeps an online-softmax state for the current (b, g) segment; when the range moves to the
 // next segment the four states are merged in shared memory into one split partial (m, l, O) of the
-// segment.  The CTA that completes a segment's ticket merges the segment's partials (same rule as
+// segment.  A second kernel, one CTA per segment, merges each segment's partials (same rule as
 // above).
 // ============================================================================================
 
@@ -382,44 +383,19 @@ struct StreamSmem {
     alignas(1024) unsigned char v[NS][DC * KV_CHUNK];
     float ob[16][D + 8];       // consumer warps' O merged at a flush (rows padded: no bank conflicts)
     float mw[kStreamConsumers][16], lw[kStreamConsumers][16];
-    int lastf[32];             // tickets taken: this CTA merges the segment
-    int fslot[32][4];          // slots of the partials of segments merged on the few-partial path
-    int flist[32], nfl;        // those segments (positions in the current group of 32)
     alignas(8) uint64_t full[NS], empty[NS];
     int js[NS];
     int32_t row[256];     // sanitised block list of the producer's current (b, g)
     int fail;
-    int last;
 };
 
 struct StreamBufs {
     float *pm;                      // [n_ctas, max_seg, 16]  running max (log2 units)
     float *pl;                      // [n_ctas, max_seg, 16]  running sum
     float *po;                      // [n_ctas, max_seg, 16, D] unnormalised output
-    unsigned long long *tickets;    // [batch * Hkv]: (call generation << 32) | partials merged
     int max_seg;
     int per_cta;                    // items per CTA (the last CTA may have fewer)
-    uint32_t gen;                   // this call's generation (never 0)
 };
-
-// Merge tickets are 64-bit words (call generation << 32) | partials counted.  A call leaves every
-// ticket it used at 0 (the CTA that merges a segment clears its ticket).  Every CTA joins the
-// tickets of its segments when it starts: a word tagged with another generation (0 after a
-// completed call, or anything in a fresh workspace) is reset to (gen, 0); once any CTA of this call
-// has joined, the tag matches and the word is not reset again.  A CTA adds its partial only after
-// its own join, so no count of this call is lost, and taking a ticket at the end is a single atomic
-// add.  (A CUDA graph replays one generation; the clearing is what makes the next replay start
-// afresh.)
-__device__ __forceinline__ void join_ticket(unsigned long long *t, uint32_t gen) {
-    unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(t);
-    while ((uint32_t)(cur >> 32) != gen) {
-        const unsigned long long seen = atomicCAS(t, cur, (unsigned long long)gen << 32);
-        if (seen == cur) break;
-        cur = seen;
-    }
-}
-// Partials counted before this one.
-__device__ __forceinline__ uint32_t take_ticket(unsigned long long *t) { return (uint32_t)atomicAdd(t, 1ull); }
 
 __device__ __forceinline__ void consumers_sync() {   // the four consumer warps only
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kStreamConsumers) : "memory");
@@ -444,7 +420,6 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
     const int n = x1 - x0;
     const int k_tot = P.k_tot;
     const int bg_first = x0 / k_tot, a_first = x0 - bg_first * k_tot;
-    const int nseg = n > 0 ? (x1 - 1) / k_tot - bg_first + 1 : 0;
     volatile int &fail = S.fail;
 
     if (warp == kStreamConsumers && lane == 0) {
@@ -591,24 +566,31 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
                 W.pl[slot + tid] = L;
             }
             // warps add their rows in a fixed order (warp 0 stores, then 1, 2, 3 add), so the
-            // partial does not depend on timing
+            // partial does not depend on timing; an adding warp reads eight columns' worth of its
+            // rows before it writes any of them back, so the shared-memory reads overlap
 #pragma unroll 1
             for (int w = 0; w < kStreamConsumers; ++w) {
                 if (w > 0) consumers_sync();
                 if (warp != w) continue;
+                constexpr int kB = D / 8 < 8 ? D / 8 : 8;
 #pragma unroll
-                for (int dt = 0; dt < D / 8; ++dt) {
-                    const int col = dt * 8 + 2 * (lane & 3);
-                    float2 *a = reinterpret_cast<float2 *>(&S.ob[r0][col]);
-                    float2 *c = reinterpret_cast<float2 *>(&S.ob[r0 + 8][col]);
-                    const float2 va = make_float2(o[dt][0] * f0, o[dt][1] * f0);
-                    const float2 vc = make_float2(o[dt][2] * f1, o[dt][3] * f1);
-                    if (w == 0) {
-                        if (r0 < P.G) *a = va;
-                        if (r0 + 8 < P.G) *c = vc;
-                    } else {
-                        if (r0 < P.G) *a = make_float2(a->x + va.x, a->y + va.y);
-                        if (r0 + 8 < P.G) *c = make_float2(c->x + vc.x, c->y + vc.y);
+                for (int d0 = 0; d0 < D / 8; d0 += kB) {
+                    float2 pa[kB], pc[kB];
+#pragma unroll
+                    for (int t = 0; t < kB; ++t) {   // rows 0..15 are all in the buffer: read freely
+                        const int col = (d0 + t) * 8 + 2 * (lane & 3);
+                        pa[t] = w == 0 ? make_float2(0.f, 0.f) : *reinterpret_cast<const float2 *>(&S.ob[r0][col]);
+                        pc[t] = w == 0 ? make_float2(0.f, 0.f) : *reinterpret_cast<const float2 *>(&S.ob[r0 + 8][col]);
+                    }
+#pragma unroll
+                    for (int t = 0; t < kB; ++t) {
+                        const int dt = d0 + t, col = dt * 8 + 2 * (lane & 3);
+                        if (r0 < P.G)
+                            *reinterpret_cast<float2 *>(&S.ob[r0][col]) =
+                                make_float2(pa[t].x + o[dt][0] * f0, pa[t].y + o[dt][1] * f0);
+                        if (r0 + 8 < P.G)
+                            *reinterpret_cast<float2 *>(&S.ob[r0 + 8][col]) =
+                                make_float2(pc[t].x + o[dt][2] * f1, pc[t].y + o[dt][3] * f1);
                     }
                 }
             }
@@ -640,8 +622,6 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
         int cur = 0;
         reset();
         if (n > 0) load_q(bg_first);
-        if (warp == 1)
-            for (int sg = lane; sg < nseg; sg += 32) join_ticket(&W.tickets[bg_first + sg], W.gen);
         int seg = 0, a = a_first;   // item x0 + k is slot a of row bg_first + seg
         for (int k = 0; k < n; ++k, a = (a + 1 == k_tot) ? 0 : a + 1, seg += (a == 0)) {
             const int s = k % NS;
@@ -741,229 +721,96 @@ __global__ void __launch_bounds__(32 * (kStreamConsumers + 1), 2) decode_stream_
         if (n > 0) flush(cur);
     }
 
-    // every partial of this CTA is written: take the tickets of its segments (up to 32 at a time,
-    // in parallel); the CTA that completes a segment merges it.  The merge issues its global loads
-    // in two rounds (the partials' maxima and sums, then their O rows), chunks of kPC partials at
-    // a time.  Shared memory reused (the loop is over): S.row -> slot of each partial, S.mw[0] /
-    // S.lw[0] -> the segment's running max and sum per row, S.ob -> per chunk the partials' maxima
-    // (then weights 2^(m_p - m) / l) and sums.
-    __threadfence();
-    __syncthreads();
-    constexpr int kPC = 32;
-    constexpr int kFewParts = 4;
-    constexpr int kThreads = 32 * (kStreamConsumers + 1);
-    constexpr int kAcc = (16 * D / 4 + kThreads - 1) / kThreads;
-    static_assert(2 * kPC * 16 <= 16 * (D + 8), "merge chunk must fit the flush buffer");
-    int *slot_of = S.row;
-    float *pm_s = &S.ob[0][0];
-    float *pl_s = pm_s + kPC * 16;
-    const int G = P.G;
-    for (int s0 = 0; s0 < nseg; s0 += 32) {
-        if (tid < min(32, nseg - s0)) {
-            const int bg = bg_first + s0 + tid;
-            const int c_first = bg * k_tot / per, c_last = ((bg + 1) * k_tot - 1) / per;
-            S.lastf[tid] = take_ticket(&W.tickets[bg]) == (uint32_t)(c_last - c_first);
-        }
-        __syncthreads();
-        // segments with at most kFewParts partials: their slots are listed first, then every
-        // thread loads the maxima, sums and O rows of its (segment, 4 columns) pairs in one round
-        // and combines them in registers, several segments per pass
-        const int ng = min(32, nseg - s0);
-        if (tid < ng) {
-            const int bg = bg_first + s0 + tid;
-            const int c_first = bg * k_tot / per;
-            const int np = ((bg + 1) * k_tot - 1) / per - c_first + 1;
-#pragma unroll
-            for (int p = 0; p < kFewParts; ++p) {
-                const int cc = c_first + min(p, np - 1);
-                S.fslot[tid][p] = p < np ? (cc * W.max_seg + (bg - cc * per / k_tot)) * 16 : -1;
-            }
-        }
-        if (tid == 0) {
-            int m = 0;
-            for (int t = 0; t < ng; ++t) {
-                const int bg = bg_first + s0 + t;
-                const int np = ((bg + 1) * k_tot - 1) / per - bg * k_tot / per + 1;
-                if (S.lastf[t] && np <= kFewParts) S.flist[m++] = t;
-            }
-            S.nfl = m;
-        }
-        __syncthreads();
-        if (S.nfl > 0) __threadfence();
-        const int per_seg4 = G * D / 4;
-        const int fb = max(1, (kAcc * kThreads) / per_seg4);
-        for (int f0 = 0; f0 < S.nfl; f0 += fb) {
-            const int pairs = min(fb, S.nfl - f0) * per_seg4;
-#pragma unroll
-            for (int u = 0; u < kAcc; ++u) {
-                const int q = tid + u * kThreads;
-                if (q < pairs) {
-                    const int t = S.flist[f0 + q / per_seg4], e4 = q % per_seg4;
-                    const int bg = bg_first + s0 + t;
-                    const int r = (e4 * 4) / D, col = (e4 * 4) % D;
-                    float mm[kFewParts], ll[kFewParts];
-                    float4 vv[kFewParts];
-#pragma unroll
-                    for (int p = 0; p < kFewParts; ++p) {
-                        const int sl = S.fslot[t][p];
-                        if (sl >= 0) {
-                            mm[p] = __ldcg(&W.pm[sl + r]);
-                            ll[p] = __ldcg(&W.pl[sl + r]);
-                            vv[p] = __ldcg(reinterpret_cast<const float4 *>(W.po + (int64_t)(sl + r) * D + col));
-                        } else {
-                            mm[p] = -INFINITY;
-                            ll[p] = 0.f;
-                            vv[p] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        }
-                    }
-                    float M = -INFINITY;
-#pragma unroll
-                    for (int p = 0; p < kFewParts; ++p) M = fmaxf(M, mm[p]);
-                    float L = 0.f;
-                    float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                    for (int p = 0; p < kFewParts; ++p) {
-                        const float f = mm[p] > -INFINITY ? ex2_approx(mm[p] - M) : 0.f;
-                        L += ll[p] * f;
-                        a4.x += vv[p].x * f;
-                        a4.y += vv[p].y * f;
-                        a4.z += vv[p].z * f;
-                        a4.w += vv[p].w * f;
-                    }
-                    const float inv = L > 0.f ? 1.f / L : 0.f;
-                    const int b = bg / P.Hkv, g = bg - b * P.Hkv;
-                    const int64_t orow = (int64_t)b * P.Hq + (int64_t)g * G + r;
-                    uint2 pk;
-                    pk.x = pack_bf16(a4.x * inv, a4.y * inv);
-                    pk.y = pack_bf16(a4.z * inv, a4.w * inv);
-                    *reinterpret_cast<uint2 *>(O + orow * D + col) = pk;
-                    if (lse && col == 0)
-                        lse[orow] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
-                    if (e4 == 0) W.tickets[bg] = 0ull;   // merged: leave the ticket clear
-                }
-            }
-        }
-        // segments with more partials: chunked, two rounds each
-        for (int seg = s0; seg < s0 + ng; ++seg) {
-            if (!S.lastf[seg - s0]) continue;   // uniform across the CTA
-            const int bg = bg_first + seg;
-            const int c_first = bg * k_tot / per;
-            const int np = ((bg + 1) * k_tot - 1) / per - c_first + 1;
-            if (np <= kFewParts) continue;      // merged above
-            __threadfence();
-            const int b = bg / P.Hkv, g = bg - b * P.Hkv;
-            for (int p = tid; p < np; p += kThreads) {
-                const int cc = c_first + p;
-                slot_of[p] = (cc * W.max_seg + (bg - cc * per / k_tot)) * 16;
-            }
-            if (tid < G) {
-                S.mw[0][tid] = -INFINITY;
-                S.lw[0][tid] = 0.f;
-            }
-            // round 1: running max and sum over the partials, chunk by chunk
-            for (int c0 = 0; c0 < np; c0 += kPC) {
-                const int cn = min(kPC, np - c0);
-                __syncthreads();
-                for (int e = tid; e < cn * G; e += kThreads) {
-                    const int q = e / G, r = e % G;
-                    const int sl = slot_of[c0 + q] + r;
-                    pm_s[q * 16 + r] = __ldcg(&W.pm[sl]);
-                    pl_s[q * 16 + r] = __ldcg(&W.pl[sl]);
-                }
-                __syncthreads();
-                if (tid < G) {
-                    float M = S.mw[0][tid], L = S.lw[0][tid];
-                    float cm = -INFINITY;
-                    for (int q = 0; q < cn; ++q) cm = fmaxf(cm, pm_s[q * 16 + tid]);
-                    if (cm > -INFINITY) {
-                        const float Mn = fmaxf(M, cm);
-                        L = (M > -INFINITY) ? L * ex2_approx(M - Mn) : 0.f;
-                        for (int q = 0; q < cn; ++q) {
-                            const float mm = pm_s[q * 16 + tid];
-                            if (mm > -INFINITY) L += pl_s[q * 16 + tid] * ex2_approx(mm - Mn);
-                        }
-                        M = Mn;
-                    }
-                    S.mw[0][tid] = M;
-                    S.lw[0][tid] = L;
-                }
-            }
-            // round 2: O = sum_p w_p O_p, w_p = 2^(m_p - m) / l
-            float4 acc[kAcc];
-#pragma unroll
-            for (int u = 0; u < kAcc; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int c0 = 0; c0 < np; c0 += kPC) {
-                const int cn = min(kPC, np - c0);
-                __syncthreads();
-                if (np > kPC) {   // segments over more than kPC CTAs: reload this chunk's maxima
-                    for (int e = tid; e < cn * G; e += kThreads) {
-                        const int q = e / G, r = e % G;
-                        pm_s[q * 16 + r] = __ldcg(&W.pm[slot_of[c0 + q] + r]);
-                    }
-                    __syncthreads();
-                }
-                if (tid < G) {
-                    const float M = S.mw[0][tid], L = S.lw[0][tid];
-                    for (int q = 0; q < cn; ++q) {
-                        const float mm = pm_s[q * 16 + tid];
-                        pm_s[q * 16 + tid] = (mm > -INFINITY && L > 0.f) ? ex2_approx(mm - M) / L : 0.f;
-                    }
-                }
-                __syncthreads();
-                for (int q0 = 0; q0 < cn; q0 += 4) {
-                    float4 v[kAcc][4];
-#pragma unroll
-                    for (int u = 0; u < kAcc; ++u) {
-                        const int e4 = tid + u * kThreads;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            v[u][q] = make_float4(0.f, 0.f, 0.f, 0.f);
-                            if (e4 * 4 < G * D && q0 + q < cn) {
-                                const int r = (e4 * 4) / D, col = (e4 * 4) % D;
-                                v[u][q] = __ldcg(reinterpret_cast<const float4 *>(
-                                    W.po + (int64_t)(slot_of[c0 + q0 + q] + r) * D + col));
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < kAcc; ++u) {
-                        const int e4 = tid + u * kThreads;
-                        if (e4 * 4 < G * D) {
-                            const int r = (e4 * 4) / D;
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const float wv = q0 + q < cn ? pm_s[(q0 + q) * 16 + r] : 0.f;
-                                acc[u].x += wv * v[u][q].x;
-                                acc[u].y += wv * v[u][q].y;
-                                acc[u].z += wv * v[u][q].z;
-                                acc[u].w += wv * v[u][q].w;
-                            }
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kAcc; ++u) {
-                const int e4 = tid + u * kThreads;
-                if (e4 * 4 < G * D) {
-                    const int r = (e4 * 4) / D, col = (e4 * 4) % D;
-                    const int64_t orow = (int64_t)b * P.Hq + (int64_t)g * G + r;
-                    uint2 pk;
-                    pk.x = pack_bf16(acc[u].x, acc[u].y);
-                    pk.y = pack_bf16(acc[u].z, acc[u].w);
-                    *reinterpret_cast<uint2 *>(O + orow * D + col) = pk;
-                    if (lse && col == 0) {
-                        const float M = S.mw[0][r], L = S.lw[0][r];
-                        lse[orow] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
-                    }
-                }
-            }
-            if (tid == 0) W.tickets[bg] = 0ull;   // merged: leave the ticket clear
-            __syncthreads();   // shared scratch free for the next segment
-        }
-        __syncthreads();       // lastf free for the next group
-    }
     if (S.fail && tid == 0) report(P.err, kErrTimeout);
+}
+
+// One CTA per (b, g) segment, one thread per 4 output columns of the segment's G query rows:
+// merges the segment's split partials, O = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p, in
+// ascending partial order.  Launched right behind the streaming kernel; griddep_wait holds it until
+// every partial is written.  The maxima and sums of all partials and the first kMergeBatch partials'
+// O columns are loaded in one round.
+constexpr int kMergeBatch = 8;
+constexpr int kMaxParts = 256;     // partials of a segment: at most k_tot <= 256
+
+template <int D>
+__global__ void __launch_bounds__(512, 1) decode_merge_kernel(Prob P, StreamBufs W, __nv_bfloat16 *__restrict__ O,
+                                                           float *__restrict__ lse) {
+    __shared__ float wsm[kMaxParts][16];   // partial maxima, then weights 2^(m_p - M) / L
+    __shared__ float lsm[kMaxParts][16];   // partial sums
+    __shared__ float Ms[16], Ls[16];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const int bg = blockIdx.x, k_tot = P.k_tot, per = W.per_cta, G = P.G;
+    griddep_launch();
+    const int c_first = bg * k_tot / per;
+    const int np = ((bg + 1) * k_tot - 1) / per - c_first + 1;
+    auto slot = [&](int p) {
+        const int cc = c_first + p;
+        return (int64_t)(cc * W.max_seg + (bg - cc * per / k_tot)) * 16;
+    };
+    const bool col_ok = tid * 4 < G * D;
+    const int r = (tid * 4) / D, col = (tid * 4) % D;
+    griddep_wait();
+    float4 v[kMergeBatch];
+#pragma unroll
+    for (int q = 0; q < kMergeBatch; ++q)
+        v[q] = (col_ok && q < np) ? __ldcg(reinterpret_cast<const float4 *>(W.po + (slot(q) + r) * D + col))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = tid; e < np * 16; e += blockDim.x) {
+        const int p = e >> 4, rr = e & 15;
+        const int64_t sl = slot(p) + rr;
+        wsm[p][rr] = __ldcg(&W.pm[sl]);
+        lsm[p][rr] = __ldcg(&W.pl[sl]);
+    }
+    __syncthreads();
+    for (int rr = warp; rr < G; rr += nw) {
+        float M = -INFINITY;
+        for (int p = lane; p < np; p += 32) M = fmaxf(M, wsm[p][rr]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+        if (M > -INFINITY)
+            for (int p = lane; p < np; p += 32) {
+                const float mm = wsm[p][rr];
+                if (mm > -INFINITY) L += lsm[p][rr] * ex2_approx(mm - M);
+            }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        __syncwarp();
+        for (int p = lane; p < np; p += 32) {
+            const float mm = wsm[p][rr];
+            wsm[p][rr] = (mm > -INFINITY && L > 0.f) ? ex2_approx(mm - M) / L : 0.f;
+        }
+        if (lane == 0) {
+            Ms[rr] = M;
+            Ls[rr] = L;
+        }
+    }
+    __syncthreads();
+    if (!col_ok) return;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p0 = 0; p0 < np; p0 += kMergeBatch) {
+        if (p0 > 0) {
+#pragma unroll
+            for (int q = 0; q < kMergeBatch; ++q)
+                v[q] = p0 + q < np ? __ldcg(reinterpret_cast<const float4 *>(W.po + (slot(p0 + q) + r) * D + col))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int q = 0; q < kMergeBatch; ++q) {
+            const float wv = p0 + q < np ? wsm[p0 + q][r] : 0.f;
+            acc.x = fmaf(wv, v[q].x, acc.x);
+            acc.y = fmaf(wv, v[q].y, acc.y);
+            acc.z = fmaf(wv, v[q].z, acc.z);
+            acc.w = fmaf(wv, v[q].w, acc.w);
+        }
+    }
+    const int b = bg / P.Hkv, g = bg - b * P.Hkv;
+    const int64_t orow = (int64_t)b * P.Hq + (int64_t)g * G + r;
+    uint2 pk;
+    pk.x = pack_bf16(acc.x, acc.y);
+    pk.y = pack_bf16(acc.z, acc.w);
+    *reinterpret_cast<uint2 *>(O + orow * D + col) = pk;
+    if (lse && col == 0) lse[orow] = Ls[r] > 0.f ? (Ms[r] + __log2f(Ls[r])) * 0.69314718055994531f : -INFINITY;
 }
 
 template <int D, int BLK>
@@ -995,8 +842,7 @@ size_t decode_stream_ws_bytes(const Prob &P, int num_sms) {
     decode_stream_geometry(P, num_sms, n_ctas, per_cta, max_seg);
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
     const size_t rows = (size_t)n_ctas * max_seg * 16;
-    return 2 * a(sizeof(float) * rows) + a(sizeof(float) * rows * P.D) +
-           a(sizeof(unsigned long long) * P.batch * P.Hkv);
+    return 2 * a(sizeof(float) * rows) + a(sizeof(float) * rows * P.D);
 }
 
 template <int D, int BLK>
@@ -1008,8 +854,12 @@ static cudaError_t launch_stream_t(const Prob &P, const CUtensorMap &tk, const C
     auto kern = decode_stream_kernel<D, BLK, NS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(n_ctas), dim3(32 * (kStreamConsumers + 1)), smem, st, P, tk, tv,
-                      (const __nv_bfloat16 *)q, block_idx, W, (__nv_bfloat16 *)O, lse);
+    e = launch_pdl(kern, dim3(n_ctas), dim3(32 * (kStreamConsumers + 1)), smem, st, P, tk, tv,
+                   (const __nv_bfloat16 *)q, block_idx, W, (__nv_bfloat16 *)O, lse);
+    if (e != cudaSuccess) return e;
+    const int threads = std::max(64, (P.G * D / 4 + 31) / 32 * 32);
+    return launch_pdl(decode_merge_kernel<D>, dim3(P.batch * P.Hkv), dim3(threads), 0, st, P, W,
+                      (__nv_bfloat16 *)O, lse);
 }
 
 cudaError_t launch_decode_stream(const Prob &P, const CUtensorMap &tk, const CUtensorMap &tv, const void *q,
@@ -1024,14 +874,8 @@ cudaError_t launch_decode_stream(const Prob &P, const CUtensorMap &tk, const CUt
     W.pm = reinterpret_cast<float *>(base);
     W.pl = reinterpret_cast<float *>(base + a(sizeof(float) * rows));
     W.po = reinterpret_cast<float *>(base + 2 * a(sizeof(float) * rows));
-    W.tickets = reinterpret_cast<unsigned long long *>(base + 2 * a(sizeof(float) * rows) +
-                                                       a(sizeof(float) * rows * P.D));
     W.max_seg = max_seg;
     W.per_cta = per_cta;
-    static std::atomic<uint32_t> generation{0};
-    uint32_t gen;
-    do gen = ++generation; while (gen == 0);
-    W.gen = gen;
     ProfScope prof("decode_attn", st);
     if (P.D == 128 && P.B == 64) return launch_stream_t<128, 64>(P, tk, tv, q, block_idx, W, n_ctas, O, lse, st);
     if (P.D == 128 && P.B == 128) return launch_stream_t<128, 128>(P, tk, tv, q, block_idx, W, n_ctas, O, lse, st);

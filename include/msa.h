@@ -248,8 +248,8 @@ msa_status_t msa_sparse_attn_prefill_bwd(const msa_config_t *cfg, const msa_shap
  *  Returns MSA_ERR_UNSUPPORTED (launching nothing, also on the size query) when batch x Hkv
  *  reaches 2^26, or batch x Hkv x k_tot or batch x Hkv x Lmax reaches 2^31 (the kernel indexes
  *  with 32-bit integers).  Repeated calls on the same inputs give bit-identical outputs, and the
- *  call may be captured in a CUDA graph: every replay recomputes and merges (its merge counters
- *  are left clear after each call).
+ *  call (two kernels: a streaming pass that writes split partials, then one merge per sequence and
+ *  KV head) may be captured in a CUDA graph: every replay recomputes everything.
  */
 msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *shape,
                                     const void *q, const void *k_cache, const void *v_cache,
@@ -276,8 +276,8 @@ msa_status_t msa_sparse_attn_decode(const msa_config_t *cfg, const msa_shape_t *
  *  - Set-up: the first call on a device looks up the array's device address (with that device
  *    current) and caches it; make that first call before any CUDA stream capture.
  *  - Sharing: every call on a device uses the same array, and the array keeps the last call's
- *    contents; nothing in it needs clearing between calls (its merge counters carry a per-call
- *    generation tag).  Calls that may overlap on the GPU
+ *    contents; nothing in it needs clearing between calls (every partial is written before the
+ *    merge reads it).  Calls that may overlap on the GPU
  *    -- on different streams, or from different threads -- race on it: serialise them.
  *  - Every GPU that loads the library holds the 40 MiB until the process exits.
  */
