@@ -448,7 +448,7 @@ def family_split(msa, job) -> dict:
     msa.profile_enable(False)
     fam = {}
     for f in ("block_keys", "index_scores", "select_topk", "index_topk", "prefill_lists", "prefill_attn",
-              "prefill_combine", "decode_attn"):
+              "prefill_combine", "decode_attn", "prefill_bwd"):
         t, n = msa.profile_read(f)
         if n:
             fam[f] = round(t, 3)
@@ -515,6 +515,7 @@ def secondary_measurements(args, dist, pf, x, sparse_ms, pk):
         out["dense_prefill_128k"] = {"ms": ms_dense, "tflops": dense_flops(pf.w) / (ms_dense / 1000) / 1e12,
                                      "speedup_of_sparse_step": ms_dense / sparse_ms}
         del od, ld
+    out["backward_128k"] = backward(dist, pf, x, pk)
     # decode at 128K: batch 32, each step replayed from a CUDA graph, L2 flushed between steps
     wd = WORKLOADS["decode_128k"]
     xd = make_inputs(wd, device="cuda", seed=100 + dist.rank)
@@ -544,6 +545,52 @@ def secondary_measurements(args, dist, pf, x, sparse_ms, pk):
                                     "speedup_of_sparse_attn": (msd / 5) / a_ms_launch}
         del wsb
     del xd, dc
+    torch.cuda.empty_cache()
+    return out
+
+
+def backward(dist, pf, x, pk):
+    """Gradients of the prefill attention (dQ, dK, dV over the selected blocks, selection fixed) for
+    the forward just run: a step zeroes the fp32 gradients and runs msa_sparse_attn_prefill_bwd over
+    all rows; dO is seeded N(0, 0.05^2) bf16.  Work = 10 D FLOPs per (query head, visible key): S
+    recomputed, dP, dV, dK, dQ (2.5 x the forward's 4 D)."""
+    from block_sparse_long_scores_b200 import msa
+    w = pf.w
+    T = pf.shape.total_rows
+    gen = torch.Generator(device="cuda").manual_seed(600 + dist.rank)
+    d_o = (torch.randn(pf.o.shape, generator=gen, device="cuda") * 0.05).to(torch.bfloat16)
+    dq = torch.zeros(T, w.Hq, w.D, dtype=torch.float32, device="cuda")
+    dk = torch.zeros(T, w.Hkv, w.D, dtype=torch.float32, device="cuda")
+    dv = torch.zeros_like(dk)
+    n = msa.msa_sparse_attn_prefill_bwd(pf.cfg, pf.shape, None, None, None, None, None, None, None, 0, T,
+                                        None, None, None, None)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
+
+    def step():
+        dq.zero_()
+        dk.zero_()
+        dv.zero_()
+        msa.msa_sparse_attn_prefill_bwd(pf.cfg, pf.shape, x["q"], x["k"], x["v"], pf.o, pf.lse, d_o, pf.block_idx,
+                                        0, T, dq, dk, dv, ws, pf.err)
+    ms = timed(step, 3, 1, dist) / 3
+    torch.cuda.synchronize()
+    msa.profile_reset()
+    msa.profile_enable(True)
+    step()
+    torch.cuda.synchronize()
+    msa.profile_enable(False)
+    fam = {f: round(msa.profile_read(f)[0], 3) for f in ("prefill_lists", "prefill_bwd")}
+    msa.profile_reset()
+    flops = 2.5 * selected_flops(pf)
+    kern_ms = fam["prefill_bwd"]
+    peak = float(pk["bf16_tflops_sustained"])
+    out = {"ms": ms, "tokens_per_s": dist.world * T / (ms / 1000), "flops": flops,
+           "tflops_step": flops / (ms / 1000) / 1e12, "kernel_ms_one_step": fam,
+           "roofline": {"bound": "tensor", "kernel": "sparse_prefill_bwd_kernel (mma.sync)",
+                        "achieved": flops / (kern_ms / 1000) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                        "frac": flops / (kern_ms / 1000) / 1e12 / peak, "peak_kind": "bf16 sustained"},
+           "err": int(pf.err.item()), "finite": bool(torch.isfinite(dq).all().item())}
+    del d_o, dq, dk, dv, ws
     torch.cuda.empty_cache()
     return out
 

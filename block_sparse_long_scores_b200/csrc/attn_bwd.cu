@@ -43,6 +43,24 @@ __global__ void bwd_rowdot_kernel(Prob P, const __nv_bfloat16 *__restrict__ O, c
     if (lane == 0) Dv[w] = acc;
 }
 
+// Add an m16n8 accumulator fragment (rows r and r + 8 of the lane group, columns c and c + 1) to
+// fp32 memory with 16-byte atomics: lanes t4 and t4 ^ 1 swap halves so that the even lane holds
+// four contiguous columns of row r and the odd lane four of row r + 8.  `at(row_half, col0)`
+// returns the address of the 4 columns from col0 of that row (rows the caller leaves out map to
+// nullptr).  The frame's columns start at 2 * (lane & 3).
+template <typename F>
+__device__ __forceinline__ void red_frag_v4(const float (&f)[4], float scale, F at) {
+    const int t4 = threadIdx.x & 3;
+    const bool even = (t4 & 1) == 0;
+    const float x = even ? f[2] : f[0], y = even ? f[3] : f[1];
+    const float xo = __shfl_xor_sync(0xffffffffu, x, 1), yo = __shfl_xor_sync(0xffffffffu, y, 1);
+    float *dst = even ? at(0, 2 * t4) : at(1, 2 * t4 - 2);
+    if (!dst) return;
+    const float4 v = even ? make_float4(f[0] * scale, f[1] * scale, xo * scale, yo * scale)
+                          : make_float4(xo * scale, yo * scale, f[2] * scale, f[3] * scale);
+    atomicAdd(reinterpret_cast<float4 *>(dst), v);
+}
+
 template <int D, int BLK, int G>
 struct BwdShape {
     static constexpr int NW = BLK / 16;        // warps: 16 keys of the block each
@@ -106,18 +124,15 @@ __global__ void __launch_bounds__(BwdShape<D, BLK, G>::THREADS) sparse_prefill_b
     auto flush = [&]() {
         if (cur_list < 0) return;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int64_t kpos = jb * BLK + key0 + gq + 8 * half;
-            if (kpos < len) {
-                const int64_t base = ((s0 + kpos) * P.Hkv + g) * D + 2 * t4;
-#pragma unroll
-                for (int nt = 0; nt < D / 8; ++nt) {
-                    atomicAdd(reinterpret_cast<float2 *>(W.dv + base + nt * 8),
-                              make_float2(dv[nt][2 * half], dv[nt][2 * half + 1]));
-                    atomicAdd(reinterpret_cast<float2 *>(W.dk + base + nt * 8),
-                              make_float2(dk[nt][2 * half] * P.scale, dk[nt][2 * half + 1] * P.scale));
-                }
-            }
+        for (int nt = 0; nt < D / 8; ++nt) {
+            auto addr = [&](float *out) {
+                return [&, out](int half, int c0) -> float * {
+                    const int64_t kpos = jb * BLK + key0 + gq + 8 * half;
+                    return kpos < len ? out + ((s0 + kpos) * P.Hkv + g) * D + nt * 8 + c0 : nullptr;
+                };
+            };
+            red_frag_v4(dv[nt], 1.f, addr(W.dv));
+            red_frag_v4(dk[nt], P.scale, addr(W.dk));
         }
 #pragma unroll
         for (int nt = 0; nt < D / 8; ++nt)
@@ -141,16 +156,32 @@ __global__ void __launch_bounds__(BwdShape<D, BLK, G>::THREADS) sparse_prefill_b
             for (int x = tid; x < BLK * (D / 8); x += A::THREADS) {
                 const int kk = x / (D / 8), e8 = x % (D / 8);
                 const int64_t kpos = jb * BLK + kk;
-                uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
                 if (kpos < len) {
                     const int64_t src = ((s0 + kpos) * P.Hkv + g) * D + e8 * 8;
-                    kv = *reinterpret_cast<const uint4 *>(W.k + src);
-                    vv = *reinterpret_cast<const uint4 *>(W.v + src);
+                    cp_async_16(S.k + kk * A::DS + e8 * 8, W.k + src);
+                    cp_async_16(S.v + kk * A::DS + e8 * 8, W.v + src);
+                } else {
+                    *reinterpret_cast<uint4 *>(S.k + kk * A::DS + e8 * 8) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(S.v + kk * A::DS + e8 * 8) = make_uint4(0, 0, 0, 0);
                 }
-                *reinterpret_cast<uint4 *>(S.k + kk * A::DS + e8 * 8) = kv;
-                *reinterpret_cast<uint4 *>(S.v + kk * A::DS + e8 * 8) = vv;
             }
         }
+        // the tile's Q and dO rows, copied asynchronously (all in flight together) while the
+        // per-row scalars below are read
+        for (int x = tid; x < A::ROWS * (D / 8); x += A::THREADS) {
+            const int r = x / (D / 8), e8 = x % (D / 8);
+            const int u = r / A::RPT, h = r % A::RPT;
+            if (u < td.z && h < G) {
+                const int64_t row = P.row_begin + (W.entries[td.y + u] >> 8);
+                const int64_t src = (row * P.Hq + (int64_t)g * G + h) * D + e8 * 8;
+                cp_async_16(S.q + r * A::DS + e8 * 8, W.q + src);
+                cp_async_16(S.dout + r * A::DS + e8 * 8, W.dout + src);
+            } else {
+                *reinterpret_cast<uint4 *>(S.q + r * A::DS + e8 * 8) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(S.dout + r * A::DS + e8 * 8) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        cp_async_commit();
         // the tile's query rows: slot u = row / RPT (a token), head h = row % RPT
         for (int r = tid; r < A::ROWS; r += A::THREADS) {
             const int u = r / A::RPT, h = r % A::RPT;
@@ -162,19 +193,7 @@ __global__ void __launch_bounds__(BwdShape<D, BLK, G>::THREADS) sparse_prefill_b
             S.lse2[r] = ok ? W.lse[row * P.Hq + (int64_t)g * G + h] * 1.4426950408889634f : INFINITY;
             S.dd[r] = ok ? W.dv_row[(row - P.row_begin) * P.Hq + (int64_t)g * G + h] : 0.f;
         }
-        for (int x = tid; x < A::ROWS * (D / 8); x += A::THREADS) {
-            const int r = x / (D / 8), e8 = x % (D / 8);
-            const int u = r / A::RPT, h = r % A::RPT;
-            uint4 qv = make_uint4(0, 0, 0, 0), gv = make_uint4(0, 0, 0, 0);
-            if (u < td.z && h < G) {
-                const int64_t row = P.row_begin + (W.entries[td.y + u] >> 8);
-                const int64_t src = (row * P.Hq + (int64_t)g * G + h) * D + e8 * 8;
-                qv = *reinterpret_cast<const uint4 *>(W.q + src);
-                gv = *reinterpret_cast<const uint4 *>(W.dout + src);
-            }
-            *reinterpret_cast<uint4 *>(S.q + r * A::DS + e8 * 8) = qv;
-            *reinterpret_cast<uint4 *>(S.dout + r * A::DS + e8 * 8) = gv;
-        }
+        cp_async_wait<0>();
         __syncthreads();
 
 #pragma unroll 1
@@ -274,18 +293,14 @@ __global__ void __launch_bounds__(BwdShape<D, BLK, G>::THREADS) sparse_prefill_b
                     }
                 }
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int row = r0 + rg * 16 + gq + 8 * half;
-                    const int64_t grow = S.grow[row];
-                    if (grow >= 0) {
+                for (int nt = 0; nt < NTW; ++nt)
+                    red_frag_v4(dq[nt], P.scale, [&](int half, int c0) -> float * {
+                        const int row = r0 + rg * 16 + gq + 8 * half;
+                        const int64_t grow = S.grow[row];
+                        if (grow < 0) return nullptr;
                         const int h = row % A::RPT;
-                        const int64_t base = (grow * P.Hq + (int64_t)g * G + h) * D + dg * A::DPW + 2 * t4;
-#pragma unroll
-                        for (int nt = 0; nt < NTW; ++nt)
-                            atomicAdd(reinterpret_cast<float2 *>(W.dq + base + nt * 8),
-                                      make_float2(dq[nt][2 * half] * P.scale, dq[nt][2 * half + 1] * P.scale));
-                    }
-                }
+                        return W.dq + (grow * P.Hq + (int64_t)g * G + h) * D + dg * A::DPW + nt * 8 + c0;
+                    });
             }
             __syncthreads();   // dS^T is rewritten by the next chunk
         }
