@@ -164,9 +164,9 @@ __global__ void prefill_tiles_kernel(int64_t L, int tpt, const int32_t *__restri
 
 // ------------------------------------------------------------------------- tcgen05 attention
 //
-// Warp-specialised persistent kernel; each CTA walks a contiguous range of tiles (tiles of one
-// list are adjacent, so a KV block is loaded once per CTA and list).  Roles:
-//   warp 0      producer: tile contexts and K/V blocks (TMA, once per list)
+// Warp-specialised persistent kernel; the CTAs sweep the tile list together in runs of
+// kSweepTiles consecutive tiles per CTA (a KV block is loaded once per CTA, list and run).  Roles:
+//   warp 0      producer: tile contexts and K/V blocks (TMA, once per list within a run)
 //   warps 2-3   query gather: cp.async of each token's G head rows into the swizzled operand
 //   warp 1      MMA issuer: S = Q K^T into one of 2 TMEM S buffers, O = P V into one of 2 TMEM O
 //               buffers; MMA1 of tile t+1 is issued before MMA2 of tile t
@@ -199,6 +199,7 @@ struct AttnShape {
 };
 
 constexpr int kSeqCache = 256;   // sequences whose offsets the attention kernel keeps in smem
+constexpr int kSweepTiles = 8;   // consecutive tiles per CTA in the attention kernel's sweep
 
 struct TileCtx {
     int64_t s0;        // first packed row of the block's sequence
@@ -297,10 +298,15 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
 
+    // Tile order: the CTAs sweep the (group-major) tile list together, CTA c taking tiles
+    // [c m, (c + 1) m) of every run of gridDim.x * m, so at any moment all CTAs work on a narrow
+    // window of lists of one kv group and the gathered query rows of that group stay in L2.  Tiles
+    // of a list that fall in one CTA's run share one K/V load.
     const int n_tiles = *W.n_tiles;
-    const int t_begin = (int)((int64_t)n_tiles * blockIdx.x / gridDim.x);
-    const int t_end = (int)((int64_t)n_tiles * (blockIdx.x + 1) / gridDim.x);
-    const int nt = t_end - t_begin;
+    constexpr int m = kSweepTiles;
+    const int sweep = (int)gridDim.x * m;
+    const int nt = (n_tiles / sweep) * m + min(max(n_tiles % sweep - (int)blockIdx.x * m, 0), m);
+    auto tile_of = [&](int i) { return (i / m) * sweep + (int)blockIdx.x * m + (i % m); };
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer (whole warp:
@@ -310,8 +316,8 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
         const int32_t *cub = seq_cached ? S.cu_blocks : P.cu_blocks;
         const int32_t *cus = seq_cached ? S.cu_seqlens : P.cu_seqlens;
         int4 td_cur = make_int4(0, 0, 0, 0), td_nxt = make_int4(0, 0, 0, 0);
-        if (lane < nt) td_cur = W.tiles[t_begin + lane];
-        if (32 + lane < nt) td_nxt = W.tiles[t_begin + 32 + lane];
+        if (lane < nt) td_cur = W.tiles[tile_of(lane)];
+        if (32 + lane < nt) td_nxt = W.tiles[tile_of(32 + lane)];
         auto td_at = [&](int i, int base) -> int4 {   // descriptor of tile i, chunk base = 32*floor(i/32) of cur
             const int r = i - base;
             int4 v;
@@ -339,7 +345,7 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
                     // crossing into the next chunk of 32 descriptors
                     base += 32;
                     td_cur = td_nxt;
-                    td_nxt = (base + 32 + lane < nt) ? W.tiles[t_begin + base + 32 + lane] : make_int4(0, 0, 0, 0);
+                    td_nxt = (base + 32 + lane < nt) ? W.tiles[tile_of(base + 32 + lane)] : make_int4(0, 0, 0, 0);
                 }
                 td_n = td_at(i + 1, base);
             }
