@@ -171,6 +171,42 @@ def test_prefill_k_covers_all_candidates_equals_dense():
     check_attention(od.float().cpu().numpy(), O_ref, ld.cpu().numpy(), L_ref)
 
 
+def _dense_check(w, x, r0=None, r1=None):
+    """Dense causal GQA prefill over rows [r0, r1) against the fp64 oracle; rows outside the range
+    must keep their previous contents."""
+    pf = Prefill(w, x)
+    T = pf.shape.total_rows
+    r0, r1 = (0, T) if r0 is None else (r0, r1)
+    od = torch.full_like(pf.o, float("nan"))
+    ld = torch.full_like(pf.lse, float("nan"))
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    msa.msa_dense_attn_prefill(pf.cfg, pf.shape, x["q"], x["k"], x["v"], r0, r1, od, ld, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    xc = cpu(x)
+    rows = np.arange(r0, r1)
+    O_ref, L_ref = orc.dense_attn(oracle_shape(w, xc), xc["q"], xc["k"], xc["v"], rows)
+    check_attention(od[r0:r1].float().cpu().numpy(), O_ref, ld[r0:r1].cpu().numpy(), L_ref)
+    assert torch.isnan(od[:r0]).all() and torch.isnan(od[r1:]).all()
+    assert torch.isnan(ld[:r0]).all() and torch.isnan(ld[r1:]).all()
+
+
+@pytest.mark.parametrize("gain", [1.0, 11.3137, 45.2548])
+def test_dense_prefill_128k_shape(gain):
+    # the dense baseline as the benchmarks run it (G 8, D 128, 64-token key steps): two sequences
+    # with ragged tails; with sharp logits the rows' running max outgrows the rescale slack
+    w = scaled_down(WORKLOADS["prefill_128k"], (1000, 1437))
+    x = make_inputs(w, device=DEV, seed=41, logit_gain=gain)
+    _dense_check(w, x)
+
+
+def test_dense_prefill_head_dim_64_and_row_range():
+    # D 64 with 64-token blocks (G 8), sharp logits, only rows [300, 1700) of three sequences
+    w = scaled_down(WORKLOADS["ragged_prefill"], (500, 77, 1300)).with_(B=64)
+    x = make_inputs(w, device=DEV, seed=42, logit_gain=8.0)
+    _dense_check(w, x, 300, 1700)
+
+
 def test_prefill_sink_and_zero_topk():
     for k, sink in [(0, 0), (0, 1), (3, 1)]:
         w = scaled_down(WORKLOADS["tiny_prefill"], (300, 5, 64)).with_(n_topk=k, use_sink=sink)
