@@ -242,8 +242,9 @@ __global__ void __launch_bounds__(128, 1) dense_prefill_kernel(Prob P, const __g
 // tiles of one kv head -- 2 x 128/max(G,8) consecutive tokens of one sequence, their G heads as
 // rows -- and sweeps the key blocks up to its last token once for both tiles:
 //   warp 0      producer: both Q tiles once, then K/V blocks through an NKV-stage TMA ring
-//   warp 1      MMA issuer: S_x = Q_x K_j^T into TMEM, O_x += P_x V_j (P read from TMEM), tiles
-//               interleaved so one tile's softmax runs while the other's MMAs do
+//   warp 1      MMA issuer: S_x = Q_x K_j^T into TMEM, O_x += P_x V_j (P read from TMEM), each issued
+//               as soon as it is ready (an event loop over both tiles), so one tile's softmax
+//               runs while the other's MMAs do and neither waits for the other
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one thread per row, P = 2^(s - m)
 //               written to TMEM as bf16; at the end O / l and the log-sum-exp to global memory
 // O accumulates in TMEM across all key blocks against a reference max m per row.  m is raised
@@ -411,27 +412,51 @@ __global__ void __launch_bounds__(384, 1) dense_fa_kernel(Prob P, const __grid_c
                 issue_s(0, 0);
                 issue_s(1, 0);
             }
-            for (int j = 0; ok && j < nblk; ++j) {
-#pragma unroll 1
-                for (int x = 0; x < 2; ++x) {
-                    if (!fa_wait(&S.p_full[x], j & 1, &S.fail)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t v0 = smem_u32(S.v[j % A::NKV]);
+            // Event-driven issue: whichever of the two tiles' next S = Q K^T (its S buffer read by the
+            // softmax, its K/V block landed) or next O += P V (its P written) is ready goes first, so
+            // neither tile's MMAs wait for the other tile's softmax.  A K/V block is released once
+            // both tiles' O += P V of it are issued.
+            int s_next[2] = {1, 1}, pv_next[2] = {0, 0};
+            int kv_seen = 1, kv_released = 0;
+            uint64_t t_idle = 0;
+            while (ok && (pv_next[0] < nblk || pv_next[1] < nblk)) {
+                bool prog = false;
+                if (kv_seen < nblk && mbar_test_wait(&S.kv_full[kv_seen % A::NKV], (kv_seen / A::NKV) & 1)) {
+                    ++kv_seen;
+                    prog = true;
+                }
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)   // A = P from TMEM: 8 columns hold 16 keys
-                        umma_bf16_ts(tmem + A::TMEM_O + x * D, tmem + A::TMEM_P + x * (KB / 2) + kk * 8,
-                                     sdesc(v0 + kk * 16 * 128, A::KV_CHUNK, 1024), idesc_o, (j | kk) != 0);
-                    umma_commit(&S.p_empty[x]);
-                    if (x == 1) umma_commit(&S.kv_empty[j % A::NKV]);   // both tiles done with block j
-                    if (j + 1 < nblk) {
-                        if (x == 0 && !fa_wait(&S.kv_full[(j + 1) % A::NKV], ((j + 1) / A::NKV) & 1, &S.fail)) {
-                            ok = false;
-                            break;
-                        }
-                        if (!fa_wait(&S.s_empty[x], ((j + 1) & 1) ^ 1, &S.fail)) { ok = false; break; }
+                for (int x = 0; x < 2; ++x) {
+                    const int js = s_next[x];
+                    if (js < nblk && js < kv_seen && mbar_test_wait(&S.s_empty[x], (js & 1) ^ 1)) {
                         tc_fence_after();
-                        issue_s(x, j + 1);
+                        issue_s(x, js);
+                        s_next[x] = js + 1;
+                        prog = true;
                     }
+                    const int jp = pv_next[x];
+                    if (jp < nblk && jp < s_next[x] && mbar_test_wait(&S.p_full[x], jp & 1)) {
+                        tc_fence_after();
+                        const uint32_t v0 = smem_u32(S.v[jp % A::NKV]);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)   // A = P from TMEM: 8 columns hold 16 keys
+                            umma_bf16_ts(tmem + A::TMEM_O + x * D, tmem + A::TMEM_P + x * (KB / 2) + kk * 8,
+                                         sdesc(v0 + kk * 16 * 128, A::KV_CHUNK, 1024), idesc_o, (jp | kk) != 0);
+                        umma_commit(&S.p_empty[x]);
+                        pv_next[x] = jp + 1;
+                        prog = true;
+                        const int both = pv_next[0] < pv_next[1] ? pv_next[0] : pv_next[1];
+                        for (; kv_released < both; ++kv_released) umma_commit(&S.kv_empty[kv_released % A::NKV]);
+                    }
+                }
+                if (prog) {
+                    t_idle = 0;
+                } else {
+                    if (*(volatile int *)&S.fail) { ok = false; break; }
+                    const uint64_t now = globaltimer();
+                    if (t_idle == 0) t_idle = now;
+                    else if (now - t_idle > kWaitLimitNs) { atomicExch(&S.fail, 1); ok = false; break; }
+                    __nanosleep(20);
                 }
             }
             umma_commit(&S.drain);   // arrives once every MMA issued above has completed
