@@ -174,13 +174,15 @@ def test_prefill_k_covers_all_candidates_equals_dense():
 def _dense_check(w, x, r0=None, r1=None):
     """Dense causal GQA prefill over rows [r0, r1) against the fp64 oracle; rows outside the range
     must keep their previous contents."""
-    pf = Prefill(w, x)
-    T = pf.shape.total_rows
+    cfg = msa.make_config(w.Hq, w.Hkv, w.D, w.B, w.d, w.n_topk, w.use_sink)
+    shape = msa.prefill_shape(x["cu_seqlens"].to(DEV, torch.int32).contiguous(),
+                              x["cu_blocks"].to(DEV, torch.int32).contiguous(), list(w.seqlens), w.B)
+    T = shape.total_rows
     r0, r1 = (0, T) if r0 is None else (r0, r1)
-    od = torch.full_like(pf.o, float("nan"))
-    ld = torch.full_like(pf.lse, float("nan"))
+    od = torch.full((T, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ld = torch.full((T, w.Hq), float("nan"), dtype=torch.float32, device=DEV)
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
-    msa.msa_dense_attn_prefill(pf.cfg, pf.shape, x["q"], x["k"], x["v"], r0, r1, od, ld, err)
+    msa.msa_dense_attn_prefill(cfg, shape, x["q"], x["k"], x["v"], r0, r1, od, ld, err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     xc = cpu(x)
@@ -205,6 +207,17 @@ def test_dense_prefill_head_dim_64_and_row_range():
     w = scaled_down(WORKLOADS["ragged_prefill"], (500, 77, 1300)).with_(B=64)
     x = make_inputs(w, device=DEV, seed=42, logit_gain=8.0)
     _dense_check(w, x, 300, 1700)
+
+
+@pytest.mark.parametrize("D_and_workload", [("128", "prefill_128k"), ("64", "ragged_prefill")])
+def test_dense_prefill_128_token_blocks(D_and_workload):
+    # 128-token blocks take the single-warpgroup dense kernel (the flash-attention kernel steps 64
+    # keys): head_dim 128 (a shape the sparse prefill refuses, the dense call accepts) and 64, two
+    # sequences with ragged tails, sharp logits
+    _, name = D_and_workload
+    w = scaled_down(WORKLOADS[name], (900, 1333)).with_(B=128)
+    x = make_inputs(w, device=DEV, seed=43, logit_gain=8.0)
+    _dense_check(w, x)
 
 
 def test_prefill_sink_and_zero_topk():
