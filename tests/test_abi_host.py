@@ -238,3 +238,70 @@ def test_decode_refuses_problems_beyond_32_bit_indexing(L):
     assert rc == 2
     rc, _ = _decode_ws(L, _cfg(), _decode_shape(4096, 65536))                  # 2^30 rows: accepted
     assert rc == 0
+
+
+def _bwd(L, cfg, shape, r0, r1, ptrs=None, ws=None, nbytes=0, dq=None):
+    """msa_sparse_attn_prefill_bwd with fake (never dereferenced) device pointers."""
+    p = ptrs if ptrs is not None else ctypes.c_void_p(0x100000)
+    n = ctypes.c_size_t(nbytes)
+    rc = L.msa_sparse_attn_prefill_bwd(ctypes.byref(cfg), ctypes.byref(shape), p, p, p, p, p, p, p, r0, r1,
+                                       dq if dq is not None else p, p, p, ws, ctypes.byref(n), None, None)
+    return rc, n.value
+
+
+def test_backward_workspace_query_and_validation(L):
+    # the size query launches nothing and needs no device; every bad argument is refused first
+    cfg, shape = _cfg(), _prefill_shape()
+    rc, need = _bwd(L, cfg, shape, 0, 4096, ptrs=None, ws=None)
+    assert rc == 0 and need > 4096 * 32 * 4                       # at least D = dO . O for the rows
+    rc, need_all = _bwd(L, cfg, shape, 0, 131072, ptrs=None, ws=None)
+    assert rc == 0 and need_all >= need
+    assert _bwd(L, cfg, shape, 10, 5)[0] == 1                     # row_end < row_begin
+    assert _bwd(L, cfg, shape, 0, 131073)[0] == 1                 # past the rows
+    dec = _decode_shape(4, 4096)
+    assert _bwd(L, cfg, dec, 0, 1)[0] == 1                        # prefill only
+    assert _bwd(L, _cfg(B=128), _prefill_shape(B=128), 0, 10)[0] == 2   # head_dim 128 x 128-token blocks
+    ws = ctypes.c_void_p(0x200000)
+    assert _bwd(L, cfg, shape, 0, 4096, ws=ws, nbytes=need - 1)[0] == 3                     # too small
+    assert _bwd(L, cfg, shape, 0, 4096, ws=ws, nbytes=need, dq=ctypes.c_void_p(0x100004))[0] == 1   # dq not 16-B
+    assert _bwd(L, cfg, shape, 0, 4096, ws=ctypes.c_void_p(0x200010), nbytes=need)[0] == 1  # workspace not 256-B
+    n = ctypes.c_size_t(need)
+    fake = ctypes.c_void_p(0x100000)
+    rc = L.msa_sparse_attn_prefill_bwd(ctypes.byref(cfg), ctypes.byref(shape), fake, fake, fake, fake, None, fake,
+                                       fake, 0, 4096, fake, fake, fake, ws, ctypes.byref(n), None, None)
+    assert rc == 1                                                # missing lse
+    # an empty row range with valid arguments is a no-op (nothing launched, no device needed)
+    assert _bwd(L, cfg, shape, 7, 7, ws=ws, nbytes=need)[0] == 0
+
+
+def test_fused_index_topk_validation(L):
+    # msa_index_topk is prefill-only and checks pointers, alignment and ranges before any launch
+    cfg, shape = _cfg(), _prefill_shape()
+    f = ctypes.c_void_p(0x100000)
+
+    def call(q=f, k=None, wq=f, wk=None, kidx=f, frm=0, r0=0, r1=16, bi=f, shp=shape):
+        return L.msa_index_topk(ctypes.byref(cfg), ctypes.byref(shp), q, k, wq, wk, kidx, frm, r0, r1, bi, None,
+                                None, None)
+    assert call(shp=_decode_shape(4, 4096)) == 2                   # decode: use msa_index_scores + select
+    assert call(q=None) == 1
+    assert call(k=f, wk=None) == 1                                 # keys to pool but no W_k
+    assert call(bi=ctypes.c_void_p(0x100002)) == 1                 # block_idx not 4-byte aligned
+    assert call(q=ctypes.c_void_p(0x100008)) == 1                  # q not 16-byte aligned
+    assert call(r0=5, r1=4) == 1
+    assert call(r1=131073) == 1
+    assert call(frm=-1) == 1                                       # the newest-block mode is decode-only
+    assert call(r0=9, r1=9) == 0                                   # empty range, keys precomputed: no launch
+
+
+def test_dense_prefill_validation(L):
+    cfg, shape = _cfg(), _prefill_shape()
+    f = ctypes.c_void_p(0x100000)
+
+    def call(q=f, o=f, lse=None, r0=0, r1=16, shp=shape):
+        return L.msa_dense_attn_prefill(ctypes.byref(cfg), ctypes.byref(shp), q, f, f, r0, r1, o, lse, None, None)
+    assert call(shp=_decode_shape(4, 4096)) == 1
+    assert call(q=None) == 1
+    assert call(o=ctypes.c_void_p(0x100008)) == 1                  # o not 16-byte aligned
+    assert call(lse=ctypes.c_void_p(0x100002)) == 1                # lse not 4-byte aligned
+    assert call(r0=3, r1=2) == 1
+    assert call(r0=4, r1=4) == 0                                   # empty range: nothing launched
