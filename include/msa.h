@@ -324,8 +324,9 @@ int64_t msa_launch_count(void);
 
 /*
  * Opt-in per-kernel timing for measurement tools.  While enabled, every kernel family the
- * library launches (block_keys, index_scores, select_topk, prefill_lists, prefill_attn,
- * prefill_combine, decode_attn, dense_decode, dense_prefill) is bracketed by a pair of CUDA events
+ * library launches (block_keys, index_scores, select_topk, index_topk, prefill_lists, prefill_attn,
+ * prefill_combine, prefill_bwd, decode_attn, dense_decode, dense_prefill) is bracketed by a pair of
+ * CUDA events
  * recorded on the caller's stream.  msa_profile_read waits for the recorded events and returns the
  * summed milliseconds and the number of bracketed launches of one family (NULL: all families);
  * msa_profile_reset forgets them.  Disabled by default; costs two event records per launch.
