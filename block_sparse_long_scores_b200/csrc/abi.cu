@@ -400,8 +400,6 @@ msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t 
     if ((st = check_shape(cfg, shape)) != MSA_OK) return st;
     if (shape->mode != MSA_PREFILL || !workspace_bytes) return MSA_ERR_INVALID_ARG;
     if (row_begin < 0 || row_end < row_begin || row_end > shape->total_rows) return MSA_ERR_INVALID_ARG;
-    // the prefill attention's rings of query, key/value and probability tiles must fit shared memory
-    if (cfg->head_dim == 128 && cfg->block_size == 128) return MSA_ERR_UNSUPPORTED;
     const int64_t R = row_end - row_begin;
     if (R >= ((int64_t)1 << 23) || R * cfg->num_kv_heads * (cfg->n_topk + 1 + cfg->use_sink) >= ((int64_t)1 << 31))
         return MSA_ERR_UNSUPPORTED;

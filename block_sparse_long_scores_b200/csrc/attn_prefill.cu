@@ -189,11 +189,13 @@ struct AttnShape {
     static constexpr int P_STAGE = BC * Q_CHUNK;
     // Query gathers arrive ~2 us after issue, so the ring keeps several in flight; two K/V stages
     // let the next list's block load while the current list's tiles run.
-    static constexpr int NQ = 4;
+    static constexpr int NQ = (D == 128 && BLK == 128) ? 2 : 4;   // 128-key blocks at D 128: shared memory
     static constexpr int NKV = 2;
     static constexpr int NCTX = 8;
     // TMEM columns: S 2 x BLK and O 2 x D (fp32), P 2 x BLK/2 (bf16 pairs: the A operand of O = P V)
-    static constexpr int TMEM_S0 = 0, TMEM_O0 = 2 * BLK, TMEM_P0 = 2 * BLK + 2 * D;
+    // S is double-buffered where the 512 columns allow (one buffer for 128-key blocks at D 128)
+    static constexpr int NSB = 2 * BLK + 2 * D + BLK <= 512 ? 2 : 1;
+    static constexpr int TMEM_S0 = 0, TMEM_O0 = NSB * BLK, TMEM_P0 = NSB * BLK + 2 * D;
     static constexpr int TMEM_COLS = 512;
     static_assert(TMEM_P0 + BLK <= TMEM_COLS, "TMEM budget");
 };
@@ -489,8 +491,8 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
                 const int qs = i % A::NQ;
                 if (!wait_or_fail(&S.q_full[qs], (i / A::NQ) & 1, &S.fail)) { ok = false; break; }
                 fence_async_smem();   // the gathered rows were written by cp.async (generic proxy)
-                const int ts = i & 1;
-                if (!wait_or_fail(&S.s_empty[ts], ((i >> 1) & 1) ^ 1, &S.fail)) { ok = false; break; }
+                const int ts = i % A::NSB;
+                if (!wait_or_fail(&S.s_empty[ts], ((i / A::NSB) & 1) ^ 1, &S.fail)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t q0 = smem_u32(S.q[qs]), k0 = smem_u32(S.kv[kvs][0]);
 #pragma unroll
@@ -525,8 +527,8 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
                 const int64_t pos = P.row_begin + (c.ent[u] >> 8) - c.s0;
                 if (pos / BLK == c.j) lim = (int)(pos - c.j * BLK);
             }
-            const int ts = i & 1;
-            if (!__all_sync(0xffffffffu, wait_or_fail(&S.s_full[ts], (i >> 1) & 1, &S.fail))) break;
+            const int ts = i % A::NSB, ps = i & 1;   // S buffer, P buffer
+            if (!__all_sync(0xffffffffu, wait_or_fail(&S.s_full[ts], (i / A::NSB) & 1, &S.fail))) break;
             tc_fence_after();
             const uint32_t sbase = tmem + lane_base + A::TMEM_S0 + ts * BLK;
             const bool masked = __any_sync(0xffffffffu, lim < BLK - 1);   // a local block in this warp
@@ -552,7 +554,7 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
             // S is in registers: release the TMEM buffer for the next-but-one tile's S = Q K^T
             tc_fence_before();
             mbar_arrive(&S.s_empty[ts]);
-            if (!__all_sync(0xffffffffu, wait_or_fail(&S.p_empty[ts], ((i >> 1) & 1) ^ 1, &S.fail))) break;
+            if (!__all_sync(0xffffffffu, wait_or_fail(&S.p_empty[ps], ((i >> 1) & 1) ^ 1, &S.fail))) break;
             // p = 2^(s * scale * log2 e - m); keys past the row's position get 2^-inf = 0.  Rows
             // without a token are computed too: their O is never stored.
             float l = 0.f;
@@ -573,12 +575,12 @@ __global__ void __launch_bounds__(384, 1) sparse_prefill_attn_kernel(Prob P, con
                 uint32_t pk[16];   // 32 keys of the P row as bf16 pairs (keys 2c, 2c+1 in column c)
 #pragma unroll
                 for (int x = 0; x < 16; ++x) pk[x] = pack_bf16(pv[2 * x], pv[2 * x + 1]);
-                tmem_st16(tmem + lane_base + A::TMEM_P0 + ts * (BLK / 2) + cc * 16, pk);
+                tmem_st16(tmem + lane_base + A::TMEM_P0 + ps * (BLK / 2) + cc * 16, pk);
             }
             tmem_st_wait();
             S.ml[i & 3][row] = make_float2(m2, l);
             tc_fence_before();   // P is read by the tensor core after the hand-off
-            mbar_arrive(&S.p_full[ts]);
+            mbar_arrive(&S.p_full[ps]);
             mbar_arrive(&S.ml_full[i & 3]);
         }
     } else if (warp >= 8) {
@@ -884,6 +886,7 @@ static cudaError_t prefill_one(const Prob &P, const CUtensorMap &tq, const CUten
     if (P.D == 128 && P.B == 64) { MSA_DISPATCH_G(P.G, e = launch_attn_t<128, 64, G_>(P, tq, tk, tv, W, num_sms, st)); }
     else if (P.D == 64 && P.B == 64) { MSA_DISPATCH_G(P.G, e = launch_attn_t<64, 64, G_>(P, tq, tk, tv, W, num_sms, st)); }
     else if (P.D == 64 && P.B == 128) { MSA_DISPATCH_G(P.G, e = launch_attn_t<64, 128, G_>(P, tq, tk, tv, W, num_sms, st)); }
+    else if (P.D == 128 && P.B == 128) { MSA_DISPATCH_G(P.G, e = launch_attn_t<128, 128, G_>(P, tq, tk, tv, W, num_sms, st)); }
     else return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;

@@ -200,9 +200,8 @@ msa_status_t msa_index_topk(const msa_config_t *cfg, const msa_shape_t *shape,
  *  Rows are processed in internal sub-chunks of msa_prefill_subchunk_rows() rows (16384 by
  *  default).  Workspace: two-phase (file header); it grows with (row_end - row_begin) up to one
  *  sub-chunk and is then two sub-chunks' worth whatever the row count.
- *  Supported (head_dim, block_size): (64, 64), (64, 128), (128, 64); (128, 128) returns
- *  MSA_ERR_UNSUPPORTED (the kernel's rings of query, key/value and probability tiles would not fit
- *  an SM's shared memory).
+ *  Supported (head_dim, block_size): (64, 64), (64, 128), (128, 64) and (128, 128) (the last with a
+ *  single S buffer in tensor memory and a two-stage query ring, to fit TMEM and shared memory).
  */
 msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t *shape,
                                      const void *q, const void *k, const void *v,
@@ -229,7 +228,8 @@ msa_status_t msa_sparse_attn_prefill(const msa_config_t *cfg, const msa_shape_t 
  *  dv the contributions of the call's rows to every key, so a prefill may be processed in row
  *  ranges.  Additions from different blocks arrive in no fixed order, so results may differ in the
  *  last bits between runs.  Workspace: two-phase, one sub-chunk's lists and per-row dot products.
- *  Supported (head_dim, block_size) as for msa_sparse_attn_prefill.
+ *  Supported (head_dim, block_size): (64, 64), (64, 128), (128, 64); (128, 128) returns
+ *  MSA_ERR_UNSUPPORTED.
  */
 msa_status_t msa_sparse_attn_prefill_bwd(const msa_config_t *cfg, const msa_shape_t *shape,
                                          const void *q, const void *k, const void *v,

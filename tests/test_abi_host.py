@@ -305,3 +305,8 @@ def test_dense_prefill_validation(L):
     assert call(lse=ctypes.c_void_p(0x100002)) == 1                # lse not 4-byte aligned
     assert call(r0=3, r1=2) == 1
     assert call(r0=4, r1=4) == 0                                   # empty range: nothing launched
+
+
+def test_prefill_accepts_head_dim_128_with_128_token_blocks(L):
+    rc, n = _ws(L, _cfg(B=128), _prefill_shape(B=128), 0, 4096)
+    assert rc == 0 and n > 0

@@ -123,6 +123,15 @@ def test_ragged_shape_sharp_logits(gain):
     _prefill_full_check(w, x, chunk_rows=1500)
 
 
+@pytest.mark.parametrize("gain", [1.0, 11.3137])
+def test_prefill_head_dim_128_with_128_token_blocks(gain):
+    # (head_dim 128, 128-token blocks): one S buffer in tensor memory and a two-stage query ring;
+    # two sequences with ragged tails, 8 scored blocks + local + sink, three chunks
+    w = scaled_down(WORKLOADS["prefill_128k"], (3000, 1777)).with_(B=128, n_topk=8)
+    x = make_inputs(w, device=DEV, seed=44, logit_gain=gain)
+    _prefill_full_check(w, x, chunk_rows=2048)
+
+
 def test_prefill_in_subchunks():
     # one attention call over 6000 rows in sub-chunks of 1000 rows: two alternating workspace halves
     w = scaled_down(WORKLOADS["prefill_128k"], (6000,))
